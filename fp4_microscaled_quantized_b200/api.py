@@ -1,0 +1,211 @@
+"""Python binding of the C-ABI library ``libfp4_b200.so`` (include/fp4.h).
+
+Argument marshalling only: torch provides device memory and the current
+stream, every computation runs in the library's CUDA kernels.  There is no
+CPU fallback -- without the built library or a CUDA device every call raises.
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfp4_b200.so")
+
+MXFP4, NVFP4 = 0, 1
+RTN, QUEST, FOUR_OVER_SIX, SR, MS_EDEN = 0, 1, 2, 3, 4
+GROUP = {MXFP4: 32, NVFP4: 16}
+
+STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED", 3: "FP4_ERR_ALIGNMENT",
+          4: "FP4_ERR_WORKSPACE", 5: "FP4_ERR_CUDA", 6: "FP4_ERR_NONFINITE_INPUT",
+          7: "FP4_ERR_TIMEOUT"}
+
+
+class Fp4Error(RuntimeError):
+    def __init__(self, status, what):
+        super().__init__("%s failed: %s (%d)" % (what, STATUS.get(status, "?"), status))
+        self.status = status
+
+
+class fp4_had(ctypes.Structure):
+    _fields_ = [("block", ctypes.c_int32), ("randomized", ctypes.c_int32),
+                ("sign_tag", ctypes.c_uint32)]
+
+
+class fp4_qtensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("scales_swz", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("mask", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load():
+    """Load the library (raises if it is missing or no CUDA device exists)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libfp4_b200.so is not built (run __graft_entry__.build())")
+    lib = ctypes.CDLL(LIB_PATH)
+    _declare(lib)
+    _lib = lib
+    return lib
+
+
+def _declare(lib):
+    P, I32, I64, U32, U64, SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32,
+                                 ctypes.c_uint64, ctypes.c_size_t)
+    QP = ctypes.POINTER(fp4_qtensor)
+    sigs = {
+        "fp4_quantize_workspace_size": (SZ, [I64, I64, I32, I32, I32]),
+        "fp4_swizzled_scale_bytes": (SZ, [I64, I64]),
+        "fp4_hadamard": (ctypes.c_int, [P, P, I64, I64, fp4_had, U64, P]),
+        "fp4_quantize": (ctypes.c_int, [P, I64, I64, I32, I32, I32, I32, fp4_had, U64, U32, QP, P, SZ, P]),
+        "fp4_requantize": (ctypes.c_int, [QP, I32, I32, fp4_had, U64, U32, QP, P, SZ, P]),
+        "fp4_swizzle_scales": (ctypes.c_int, [P, I64, I64, P, P]),
+        "fp4_get_last_error": (ctypes.c_int, [P]),
+        "fp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _declare_extra(lib)
+
+
+def _declare_extra(lib):
+    """Entry points added by later layers (GEMM, linear)."""
+    P, I32, I64, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    QP = ctypes.POINTER(fp4_qtensor)
+    extra = {
+        "fp4_gemm": (ctypes.c_int, [QP, QP, P, I32, P, I32, P, SZ, P]),
+        "fp4_gemm_workspace_size": (SZ, [I64, I64, I64]),
+    }
+    for name, (res, args) in extra.items():
+        if hasattr(lib, name):
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check(st, what):
+    if st != 0:
+        raise Fp4Error(st, what)
+
+
+@dataclass
+class QTensor:
+    """A quantised tensor in device memory (rows x cols, groups along cols)."""
+    codes: torch.Tensor                    # uint8 rows x cols/2
+    scales: Optional[torch.Tensor]         # uint8 rows x cols/g
+    scales_swz: Optional[torch.Tensor]     # uint8 tensor-core layout
+    tensor_scale: torch.Tensor             # float32 [1]
+    mask: Optional[torch.Tensor]           # uint8 rows x cols/8 (QuEST)
+    rows: int
+    cols: int
+    fmt: int
+
+    @property
+    def group(self):
+        return GROUP[self.fmt]
+
+    def c_struct(self):
+        return fp4_qtensor(self.codes.data_ptr(),
+                           self.scales.data_ptr() if self.scales is not None else 0,
+                           self.scales_swz.data_ptr() if self.scales_swz is not None else 0,
+                           self.tensor_scale.data_ptr(),
+                           self.mask.data_ptr() if self.mask is not None else 0,
+                           self.rows, self.cols, self.fmt, 0)
+
+
+def alloc_qtensor(rows, cols, fmt, linear=True, swizzled=True, mask=False, device="cuda"):
+    lib = load()
+    g = GROUP[fmt]
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+    sc = torch.empty((rows, cols // g), dtype=torch.uint8, device=device) if linear else None
+    nswz = lib.fp4_swizzled_scale_bytes(rows, cols // g)
+    swz = torch.empty((max(nswz, 1),), dtype=torch.uint8, device=device) if swizzled else None
+    ts = torch.empty((1,), dtype=torch.float32, device=device)
+    mk = torch.empty((rows, cols // 8), dtype=torch.uint8, device=device) if mask else None
+    return QTensor(codes, sc, swz, ts, mk, rows, cols, fmt)
+
+
+def workspace_size(rows, cols, fmt, rnd, had_block):
+    return int(load().fp4_quantize_workspace_size(rows, cols, fmt, rnd, had_block))
+
+
+def alloc_workspace(nbytes, device="cuda"):
+    return torch.empty((max(int(nbytes), 16),), dtype=torch.uint8, device=device)
+
+
+def quantize(x, fmt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0, tensor_tag=0,
+             transpose=False, linear=True, swizzled=True, out=None, ws=None):
+    """fp4_quantize of a bf16 CUDA tensor; returns a QTensor."""
+    lib = load()
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
+    in_rows, in_cols = x.shape
+    rows, cols = (in_cols, in_rows) if transpose else (in_rows, in_cols)
+    if out is None:
+        out = alloc_qtensor(rows, cols, fmt, linear, swizzled, mask=(rnd == QUEST), device=x.device)
+    need = workspace_size(rows, cols, fmt, rnd, had_block)
+    if ws is None:
+        ws = alloc_workspace(need, x.device)
+    cs = out.c_struct()
+    st = lib.fp4_quantize(_ptr(x), in_rows, in_cols, int(transpose), fmt, rnd, GROUP[fmt],
+                          fp4_had(had_block, int(randomized), sign_tag), seed, tensor_tag,
+                          ctypes.byref(cs), _ptr(ws), ws.numel(), _stream())
+    _check(st, "fp4_quantize")
+    return out
+
+
+def requantize(qt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0, tensor_tag=0,
+               transpose=True, linear=True, swizzled=True, out=None, ws=None):
+    lib = load()
+    rows, cols = (qt.cols, qt.rows) if transpose else (qt.rows, qt.cols)
+    if out is None:
+        out = alloc_qtensor(rows, cols, qt.fmt, linear, swizzled, mask=(rnd == QUEST),
+                            device=qt.codes.device)
+    need = workspace_size(rows, cols, qt.fmt, rnd, had_block)
+    if ws is None:
+        ws = alloc_workspace(need, qt.codes.device)
+    cin, cout = qt.c_struct(), out.c_struct()
+    st = lib.fp4_requantize(ctypes.byref(cin), int(transpose), rnd,
+                            fp4_had(had_block, int(randomized), sign_tag), seed, tensor_tag,
+                            ctypes.byref(cout), _ptr(ws), ws.numel(), _stream())
+    _check(st, "fp4_requantize")
+    return out
+
+
+def hadamard(x, block, randomized=False, seed=0, sign_tag=0):
+    lib = load()
+    y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    st = lib.fp4_hadamard(_ptr(x), _ptr(y), x.shape[0], x.shape[1],
+                          fp4_had(block, int(randomized), sign_tag), seed, _stream())
+    _check(st, "fp4_hadamard")
+    return y
+
+
+def swizzle_scales(scales):
+    lib = load()
+    rows, ng = scales.shape
+    out = torch.empty((max(lib.fp4_swizzled_scale_bytes(rows, ng), 1),), dtype=torch.uint8,
+                      device=scales.device)
+    _check(lib.fp4_swizzle_scales(_ptr(scales), rows, ng, _ptr(out), _stream()), "fp4_swizzle_scales")
+    return out
+
+
+def get_last_error():
+    return int(load().fp4_get_last_error(_stream()))

@@ -1,0 +1,273 @@
+// C ABI entry points of the quantisation path (include/fp4.h): argument
+// validation, workspace layout, kernel sequencing and the device status word.
+#include <mutex>
+
+#include "../../include/fp4.h"
+#include "quant_dispatch.cuh"
+
+namespace fp4 {
+
+__device__ int g_status = 0;
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+// Address of the status word on the current device (looked up once per device).
+int* status_ptr() {
+  static std::mutex mu;
+  static int* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<int*>(a);
+  }
+  return addr[dev];
+}
+
+static inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+static inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t amax = 0, pseudo = 0, eden = 0, total = 0;
+};
+
+static WsLayout ws_layout(int64_t rows, int64_t cols, int fmt, int rnd, int had) {
+  WsLayout w;
+  if (fmt == FP4_NVFP4 && rnd == FP4_MS_EDEN && had > 0) {
+    w.amax = 0;
+    w.pseudo = 256;
+    w.eden = w.pseudo + align256(size_t(rows) * size_t(cols / 16) * 2);
+    w.total = w.eden + align256(size_t(rows) * size_t(cols / had) * 4);
+  } else if (fmt == FP4_NVFP4) {
+    w.total = 256;
+  }
+  return w;
+}
+
+static bool combo_supported(int fmt, int rnd, int had) {
+  if (had != 0 && had != 16 && had != 32 && had != 128) return false;
+  if (fmt == FP4_MXFP4 && (rnd == FP4_FOUR_OVER_SIX || rnd == FP4_MS_EDEN)) return false;
+  int g = fmt == FP4_NVFP4 ? 16 : 32;
+  if (rnd == FP4_MS_EDEN && (had == 0 || had < g)) return false;
+  return true;
+}
+
+static int check_out(const fp4_qtensor* out) {
+  if (!out || !out->codes || !out->tensor_scale || (!out->scales && !out->scales_swz))
+    return FP4_ERR_INVALID_ARG;
+  if (!aligned(out->codes, 16) || (out->scales_swz && !aligned(out->scales_swz, 16)) ||
+      !aligned(out->tensor_scale, 4))
+    return FP4_ERR_ALIGNMENT;
+  return FP4_OK;
+}
+
+__global__ void k_swizzle(const uint8_t* sc, int64_t rows, int64_t ng, int64_t nkb, uint8_t* swz) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < rows * ng;
+       i += int64_t(gridDim.x) * blockDim.x)
+    swz[swz_offset(i / ng, i % ng, nkb)] = sc[i];
+}
+
+static int launch_pad(uint8_t* swz, int64_t rows, int64_t ng, cudaStream_t s) {
+  int64_t nkb = (ng + 3) / 4;
+  if (!swz || ((rows % 128) == 0 && (ng % 4) == 0)) return FP4_OK;
+  int64_t n = (((rows + 127) / 128) * 128 - rows) * nkb * 4 + rows * (nkb * 4 - ng);
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  k_swz_pad<<<unsigned(blocks), 256, 0, s>>>(swz, rows, ng, nkb);
+  return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+// Shared sequencing of fp4_quantize / fp4_requantize.
+static int run_quant(int load, int fmt, int rnd, int had, QParams& p, void* ws, size_t ws_bytes,
+                     cudaStream_t s) {
+  WsLayout L = ws_layout(p.rows, p.cols, fmt, rnd, had);
+  if (L.total > 0) {
+    if (!ws || ws_bytes < L.total) return FP4_ERR_WORKSPACE;
+    if (!aligned(ws, 16)) return FP4_ERR_ALIGNMENT;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.amax_bits = L.total ? reinterpret_cast<uint32_t*>(w + L.amax) : nullptr;
+  p.pseudo = (L.pseudo ? reinterpret_cast<uint16_t*>(w + L.pseudo) : nullptr);
+  p.eden_S = (L.eden ? reinterpret_cast<float*>(w + L.eden) : nullptr);
+  p.status = status_ptr();
+  p.nkb = ((p.cols / (fmt == FP4_NVFP4 ? 16 : 32)) + 3) / 4;
+  auto launch = [&](int r) -> cudaError_t {
+    switch (load) {
+      case LD_ROW: return launch_quant<LD_ROW>(fmt, r, had, p, s);
+      case LD_TRANS: return launch_quant<LD_TRANS>(fmt, r, had, p, s);
+      case LD_ROW_FP4: return launch_quant<LD_ROW_FP4>(fmt, r, had, p, s);
+      default: return launch_quant<LD_TRANS_FP4>(fmt, r, had, p, s);
+    }
+  };
+  if (fmt == FP4_NVFP4) {
+    if (cudaMemsetAsync(p.amax_bits, 0, sizeof(uint32_t), s) != cudaSuccess) return FP4_ERR_CUDA;
+    if (rnd != FP4_MS_EDEN && launch(R_AMAX) != cudaSuccess) return FP4_ERR_CUDA;
+  }
+  if (launch(rnd) != cudaSuccess) return FP4_ERR_CUDA;
+  if (rnd == FP4_MS_EDEN) {
+    int64_t groups = p.rows * (p.cols / 16);
+    int64_t blocks = (groups + 255) / 256, cap = int64_t(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    switch (had) {
+      case 16: k_eden_pass2<16><<<unsigned(blocks), 256, 0, s>>>(p); break;
+      case 32: k_eden_pass2<32><<<unsigned(blocks), 256, 0, s>>>(p); break;
+      default: k_eden_pass2<128><<<unsigned(blocks), 256, 0, s>>>(p); break;
+    }
+    if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
+  }
+  return launch_pad(p.swz, p.rows, p.cols / (fmt == FP4_NVFP4 ? 16 : 32), s);
+}
+
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" {
+
+size_t fp4_quantize_workspace_size(int64_t rows, int64_t cols, int32_t fmt, int32_t rounding,
+                                   int32_t had_block) {
+  if (rows < 0 || cols < 0) return 0;
+  return ws_layout(rows, cols, fmt, rounding, had_block).total;
+}
+
+size_t fp4_swizzled_scale_bytes(int64_t rows, int64_t n_groups) {
+  if (rows <= 0 || n_groups <= 0) return 0;
+  return size_t((rows + 127) / 128) * size_t((n_groups + 3) / 4) * 512;
+}
+
+int fp4_quantize(const void* x, int64_t in_rows, int64_t in_cols, int32_t transpose, int32_t fmt,
+                 int32_t rounding, int32_t group, fp4_had had, uint64_t seed, uint32_t tensor_tag,
+                 fp4_qtensor* out, void* ws, size_t ws_bytes, fp4_stream_t stream) {
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (rounding < FP4_RTN || rounding > FP4_MS_EDEN) return FP4_ERR_INVALID_ARG;
+  const int g = fmt == FP4_NVFP4 ? 16 : 32;
+  if (group != g) return FP4_ERR_UNSUPPORTED;
+  if (!combo_supported(fmt, rounding, had.block)) return FP4_ERR_UNSUPPORTED;
+  if (in_rows < 0 || in_cols < 0 || (transpose != 0 && transpose != 1) || !out)
+    return FP4_ERR_INVALID_ARG;
+  const int64_t rows = transpose ? in_cols : in_rows, cols = transpose ? in_rows : in_cols;
+  const int64_t chunk = had.block > g ? had.block : g;
+  if (cols % chunk) return FP4_ERR_INVALID_ARG;
+  if (transpose && (in_cols % 8)) return FP4_ERR_ALIGNMENT;
+  out->rows = rows; out->cols = cols; out->fmt = fmt;
+  if (rows == 0 || cols == 0) return FP4_OK;   // empty tensor: nothing to launch
+  int st = check_out(out);
+  if (st) return st;
+  if (!x) return FP4_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return FP4_ERR_ALIGNMENT;
+  QParams p{};
+  p.x = x; p.in_rows = in_rows; p.in_cols = in_cols; p.rows = rows; p.cols = cols;
+  p.codes = out->codes; p.scales = out->scales; p.swz = out->scales_swz; p.mask = out->mask;
+  p.ts = out->tensor_scale; p.seed = seed; p.tensor_tag = tensor_tag; p.sign_tag = had.sign_tag;
+  p.randomized = had.randomized ? 1 : 0;
+  return run_quant(transpose ? LD_TRANS : LD_ROW, fmt, rounding, had.block, p, ws, ws_bytes,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fp4_requantize(const fp4_qtensor* in, int32_t transpose, int32_t rounding, fp4_had had,
+                   uint64_t seed, uint32_t tensor_tag, fp4_qtensor* out, void* ws, size_t ws_bytes,
+                   fp4_stream_t stream) {
+  if (!in) return FP4_ERR_INVALID_ARG;
+  if ((in->rows > 0 && in->cols > 0) && (!in->codes || !in->scales || !in->tensor_scale))
+    return FP4_ERR_INVALID_ARG;
+  if (in->fmt != FP4_MXFP4 && in->fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (rounding < FP4_RTN || rounding > FP4_MS_EDEN || (transpose != 0 && transpose != 1))
+    return FP4_ERR_INVALID_ARG;
+  const int fmt = in->fmt, g = fmt == FP4_NVFP4 ? 16 : 32;
+  if (!combo_supported(fmt, rounding, had.block)) return FP4_ERR_UNSUPPORTED;
+  if (in->rows < 0 || in->cols < 0 || in->cols % g || !out) return FP4_ERR_INVALID_ARG;
+  const int64_t rows = transpose ? in->cols : in->rows, cols = transpose ? in->rows : in->cols;
+  const int64_t chunk = had.block > g ? had.block : g;
+  if (cols % chunk) return FP4_ERR_INVALID_ARG;
+  if (transpose && (in->cols % 16)) return FP4_ERR_ALIGNMENT;
+  out->rows = rows; out->cols = cols; out->fmt = fmt;
+  if (rows == 0 || cols == 0) return FP4_OK;
+  int st = check_out(out);
+  if (st) return st;
+  if (!aligned(in->codes, 16)) return FP4_ERR_ALIGNMENT;
+  QParams p{};
+  p.x = in->codes; p.in_scales = in->scales; p.in_ts = in->tensor_scale; p.in_fmt = fmt;
+  p.in_rows = in->rows; p.in_cols = in->cols; p.rows = rows; p.cols = cols;
+  p.codes = out->codes; p.scales = out->scales; p.swz = out->scales_swz; p.mask = out->mask;
+  p.ts = out->tensor_scale; p.seed = seed; p.tensor_tag = tensor_tag; p.sign_tag = had.sign_tag;
+  p.randomized = had.randomized ? 1 : 0;
+  return run_quant(transpose ? LD_TRANS_FP4 : LD_ROW_FP4, fmt, rounding, had.block, p, ws,
+                   ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fp4_hadamard(const void* x, float* y, int64_t rows, int64_t cols, fp4_had had, uint64_t seed,
+                 fp4_stream_t stream) {
+  if (had.block != 16 && had.block != 32 && had.block != 128) return FP4_ERR_UNSUPPORTED;
+  if (rows < 0 || cols < 0 || cols % had.block) return FP4_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return FP4_OK;
+  if (!x || !y) return FP4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16)) return FP4_ERR_ALIGNMENT;
+  QParams p{};
+  p.x = x; p.rows = rows; p.cols = cols; p.seed = seed; p.sign_tag = had.sign_tag;
+  p.randomized = had.randomized ? 1 : 0;
+  int64_t tasks = rows * (cols / 8), blocks = (tasks + 255) / 256, cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (had.block) {
+    case 16: k_hadamard<16><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
+    case 32: k_hadamard<32><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
+    default: k_hadamard<128><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+int fp4_swizzle_scales(const uint8_t* scales, int64_t rows, int64_t n_groups, uint8_t* swz,
+                       fp4_stream_t stream) {
+  if (rows < 0 || n_groups < 0) return FP4_ERR_INVALID_ARG;
+  if (rows == 0 || n_groups == 0) return FP4_OK;
+  if (!scales || !swz) return FP4_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int64_t nkb = (n_groups + 3) / 4, n = rows * n_groups, blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  k_swizzle<<<unsigned(blocks), 256, 0, s>>>(scales, rows, n_groups, nkb, swz);
+  if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
+  return launch_pad(swz, rows, n_groups, s);
+}
+
+int fp4_get_last_error(fp4_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FP4_ERR_CUDA;
+  int* a = status_ptr();
+  if (!a) return FP4_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, a, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FP4_ERR_CUDA;
+  if (v) {
+    int z = 0;
+    cudaMemcpy(a, &z, sizeof(int), cudaMemcpyHostToDevice);
+  }
+  return v;
+}
+
+const char* fp4_status_string(int st) {
+  switch (st) {
+    case FP4_OK: return "ok";
+    case FP4_ERR_INVALID_ARG: return "invalid argument";
+    case FP4_ERR_UNSUPPORTED: return "unsupported combination";
+    case FP4_ERR_ALIGNMENT: return "misaligned pointer or dimension";
+    case FP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case FP4_ERR_CUDA: return "CUDA error";
+    case FP4_ERR_NONFINITE_INPUT: return "non-finite input";
+    case FP4_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

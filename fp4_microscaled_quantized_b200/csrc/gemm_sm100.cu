@@ -1,0 +1,482 @@
+// Block-scaled FP4 GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// D[M x N] = (A . SFA) (B . SFB)^T * (tA * tB), both operands K-major ("TN"),
+// FP32 accumulation in tensor memory -- the Quartet page's stage-2 kernel
+// D = C + (A x SFA) . (B x SFB); NVFP4 uses kind::mxf4nvf4 with E4M3 scales per
+// 16, MXFP4 kind::mxf4 with E8M0 scales per 32.  An optional epilogue applies
+// the Quartet backward correction dx = 16/9 H32^-1(dx_q (.) (1 - M)) (the 16/9
+// is the product of the two 4/3 tensor scales).
+//
+// Structure: persistent CTAs (one per SM), 128 x 256 output tiles, a 4-stage
+// shared-memory ring fed by TMA (codes, 128-byte swizzle) and bulk copies
+// (scale atoms, already in the tensor-core layout), warp roles:
+//   warp 0  TMA producer          warp 1  MMA issuer (one thread)
+//   warp 2  TMEM allocator        warps 4-7  epilogue (TMEM -> registers -> HBM)
+// Every mbarrier wait is bounded; on timeout the kernel records
+// FP4_ERR_TIMEOUT, stops issuing work, frees its TMEM and returns.
+#include <cuda.h>
+#include <mutex>
+
+#include "../../include/fp4.h"
+#include "device_common.cuh"
+
+namespace fp4 {
+
+int* status_ptr();
+int num_sms();
+
+namespace gemm {
+
+constexpr int BM = 128, BN = 256, BK = 256;         // BK in FP4 elements (128 bytes)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK / 2;                 // 16 KB
+constexpr int B_BYTES = BN * BK / 2;                 // 32 KB
+constexpr int SFA_BYTES = 4 * 512;                   // up to 4 atoms (NVFP4)
+constexpr int SFB_BYTES = 8 * 512;                   // 2 row blocks x 4 atoms
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int THREADS = 256;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
+constexpr unsigned long long WAIT_LIMIT = 4000000000ull;  // ~2 s of SM clocks
+
+enum : int { OUT_F32 = 0, OUT_BF16 = 1 };
+
+struct Params {
+  int64_t M, N, K;
+  const uint8_t* sfa;   // swizzled scale atoms of A
+  const uint8_t* sfb;
+  int64_t nkb;          // atoms per 128-row block (= ceil(K / g / 4))
+  const float* ta;
+  const float* tb;
+  void* D;
+  const uint8_t* mask;  // epilogue clip mask (M x N bits) or null
+  int* status;
+};
+
+// ----------------------------------------------------------- PTX helpers --
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false (and the abort flag raised) when the limit is hit.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  if (mbar_try(b, parity)) return true;
+  const unsigned long long t0 = clock64();
+  while (true) {
+    if (mbar_try(b, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > WAIT_LIMIT) {
+      *abort_flag = 1;
+      flag_status(status, ST_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// K-major operand tile with the 128-byte swizzle: 8-row core groups 1024 B
+// apart (SBO), one swizzle atom along K (LBO unused), descriptor version 1.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFF);
+  d |= uint64_t(1024 >> 4) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Scale atom source for tcgen05.cp: 32 rows x 16 bytes, no swizzle, 8-row
+// core matrices 128 B apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFF);
+  d |= uint64_t(128 >> 4) << 32;
+  d |= uint64_t(1) << 46;
+  return d;
+}
+
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+template <int FMT>
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t sfa, uint32_t sfb, uint32_t acc) {
+  if (FMT == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+        : "memory");
+  }
+}
+
+// Instruction descriptor of the block-scaled MMA: E2M1 x E2M1, both K-major,
+// N and M, scale type (0 = UE4M3, 1 = UE8M0) and the scale byte ids.
+__device__ __forceinline__ uint32_t idesc(int fmt, int n, int m, uint32_t sfa_id, uint32_t sfb_id) {
+  uint32_t d = 0;
+  d |= (sfb_id & 3u) << 4;
+  d |= 1u << 7;                    // A: E2M1
+  d |= 1u << 10;                   // B: E2M1
+  d |= uint32_t(n >> 3) << 17;
+  d |= uint32_t(fmt == 1 ? 0 : 1) << 23;
+  d |= uint32_t(m >> 4) << 24;
+  d |= (sfa_id & 3u) << 29;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Tile order: groups of 16 M-blocks sweep all N-blocks, so the CTAs resident
+// at one time share A rows and B rows in L2.
+__device__ __forceinline__ void tile_coords(int64_t t, int64_t nm, int64_t nn, int64_t& mb, int64_t& nb) {
+  const int64_t G = 16;
+  int64_t per_group = G * nn;
+  int64_t g = t / per_group, r = t % per_group;
+  int64_t gm = nm - g * G < G ? nm - g * G : G;
+  mb = g * G + r % gm;
+  nb = r / gm;
+}
+
+// ---------------------------------------------------------------- kernel --
+template <int FMT, int OUT, int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+    k_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sSFA = sB + STAGES * B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nm = (p.M + BM - 1) / BM, nn = (p.N + BN - 1) / BN, ntiles = nm * nn;
+  const int64_t nkt = (p.K + BK - 1) / BK;
+  constexpr int G = FMT == 1 ? 16 : 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 128);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer --
+    int s = 0;
+    uint32_t ph = 0;
+    for (int64_t t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      int64_t mb, nb;
+      tile_coords(t, nm, nn, mb, nb);
+      for (int64_t kt = 0; kt < nkt; ++kt) {
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.status)) break;
+        const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
+        const int n_mma = kel / 64;
+        const int atoms = FMT == 1 ? n_mma : (n_mma + 1) / 2;       // per 128-row block
+        const int64_t atom0 = kt * (BK / G / 4);
+        const int64_t nrb = (p.N + 127) / 128;
+        const int rb_b = (nb * 2 + 1 < nrb) ? 2 : 1;
+        const uint32_t sf_bytes = uint32_t(atoms) * 512u * uint32_t(1 + rb_b);
+        mbar_expect_tx(&full[s], uint32_t(A_BYTES + B_BYTES) + sf_bytes);
+        tma_load_2d(sA + s * A_BYTES, &map_a, int(kt * (BK / 2)), int(mb * BM), &full[s]);
+        tma_load_2d(sB + s * B_BYTES, &map_b, int(kt * (BK / 2)), int(nb * BN), &full[s]);
+        bulk_load(sSFA + s * SFA_BYTES, p.sfa + (mb * p.nkb + atom0) * 512, atoms * 512u, &full[s]);
+        for (int r = 0; r < rb_b; ++r)
+          bulk_load(sSFB + s * SFB_BYTES + r * 4 * 512, p.sfb + ((nb * 2 + r) * p.nkb + atom0) * 512,
+                    atoms * 512u, &full[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // --------------------------------------------------------- MMA issue --
+    int s = 0;
+    uint32_t ph = 0, acc_ph = 0;
+    for (int64_t t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+      if (!mbar_wait(acc_empty, acc_ph ^ 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      bool ok = true;
+      for (int64_t kt = 0; kt < nkt; ++kt) {
+        if (!mbar_wait(&full[s], ph, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
+        const int n_mma = kel / 64;
+        const int atoms = FMT == 1 ? n_mma : (n_mma + 1) / 2;
+        const uint32_t a_base = smem_u32(sA + s * A_BYTES), b_base = smem_u32(sB + s * B_BYTES);
+        for (int a = 0; a < atoms; ++a) {
+          tc_cp_sf(tmem + SFA_COL + 4 * a, desc_sf(smem_u32(sSFA + s * SFA_BYTES + a * 512)));
+          tc_cp_sf(tmem + SFB_COL + 8 * a, desc_sf(smem_u32(sSFB + s * SFB_BYTES + a * 512)));
+          tc_cp_sf(tmem + SFB_COL + 8 * a + 4, desc_sf(smem_u32(sSFB + s * SFB_BYTES + (4 + a) * 512)));
+        }
+        for (int kk = 0; kk < n_mma; ++kk) {
+          const int atom = FMT == 1 ? kk : kk / 2;
+          const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
+          const uint32_t sfa = (tmem + SFA_COL + 4 * atom) | (sf_id << 30);
+          const uint32_t sfb = (tmem + SFB_COL + 8 * atom) | (sf_id << 30);
+          tc_mma<FMT>(tmem + ACC_COL, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
+                      idesc(FMT, BN, BM, sf_id, sf_id), sfa, sfb, (kt > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+      if (!ok) break;
+      tc_commit(acc_full);
+      acc_ph ^= 1;
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------- epilogue --
+    const int q = warp & 3;
+    uint32_t acc_ph = 0;
+    const float tscale = __fmul_rn(*p.ta, *p.tb);
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      int64_t mb, nb;
+      tile_coords(t, nm, nn, mb, nb);
+      if (!mbar_wait(acc_full, acc_ph, abort_flag, p.status)) break;
+      acc_ph ^= 1;
+      tc_fence_after();
+      const int64_t row = mb * BM + q * 32 + lane;
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + ACC_COL + (uint32_t(q * 32) << 16) + c * 32, v);
+        const int64_t col0 = nb * BN + c * 32;
+        if (row >= p.M || col0 >= p.N) continue;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = v[j] * tscale;
+        if (EPI == 1) {
+          if (p.mask) {
+            uint32_t mw = *reinterpret_cast<const uint32_t*>(p.mask + row * (p.N >> 3) + (col0 >> 3));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if ((mw >> j) & 1u) v[j] = 0.0f;
+          }
+#pragma unroll
+          for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i & h) continue;
+              float a = v[i], b = v[i + h];
+              v[i] = a + b;
+              v[i + h] = a - b;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= 0.176776695296636881f;
+        }
+        const int ncols = int(p.N - col0 < 32 ? p.N - col0 : 32);
+        if (OUT == OUT_F32) {
+          float* dst = static_cast<float*>(p.D) + row * p.N + col0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            if (j < ncols) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        } else {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.D) + row * p.N + col0;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            if (j >= ncols) continue;
+            uint4 w;
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(v[j + 2 * i], v[j + 2 * i + 1]);
+              wp[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            *reinterpret_cast<uint4*>(dst + j) = w;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+// ------------------------------------------------------------ host side --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// Codes of a rows x K tensor as a 2-D uint8 tensor (K/2 bytes per row), box
+// 128 bytes x box_rows, 128-byte swizzle, zero fill outside.
+static bool make_map(CUtensorMap* m, const void* codes, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(K / 2), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(K / 2)};
+  cuuint32_t box[2] = {128, cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int FMT, int OUT, int EPI>
+static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+  auto kern = k_gemm<FMT, OUT, EPI>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
+  int grid = int(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace gemm
+}  // namespace fp4
+
+using namespace fp4;
+
+extern "C" int fp4_gemm(const fp4_qtensor* A, const fp4_qtensor* B, void* D, int32_t out_dtype,
+                        const uint8_t* epi_mask, int32_t epi_inverse_had, fp4_stream_t stream) {
+  if (!A || !B) return FP4_ERR_INVALID_ARG;
+  if (A->fmt != B->fmt || (A->fmt != FP4_MXFP4 && A->fmt != FP4_NVFP4)) return FP4_ERR_INVALID_ARG;
+  if (out_dtype != 0 && out_dtype != 1) return FP4_ERR_INVALID_ARG;
+  if (epi_inverse_had != 0 && epi_inverse_had != 32) return FP4_ERR_UNSUPPORTED;
+  if (epi_mask && !epi_inverse_had) return FP4_ERR_UNSUPPORTED;
+  const int64_t M = A->rows, N = B->rows, K = A->cols;
+  if (M < 0 || N < 0 || K < 0 || B->cols != K) return FP4_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP4_OK;
+  if (K % 64 || N % 8) return FP4_ERR_INVALID_ARG;
+  if (epi_inverse_had && N % 32) return FP4_ERR_INVALID_ARG;
+  if (!A->codes || !B->codes || !A->scales_swz || !B->scales_swz || !A->tensor_scale ||
+      !B->tensor_scale || !D)
+    return FP4_ERR_INVALID_ARG;
+  auto al = [](const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+  if (!al(A->codes, 16) || !al(B->codes, 16) || !al(A->scales_swz, 16) || !al(B->scales_swz, 16) ||
+      !al(D, 16) || (epi_mask && !al(epi_mask, 4)))
+    return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    size_t bytes = size_t(M) * size_t(N) * (out_dtype ? 2 : 4);
+    return cudaMemsetAsync(D, 0, bytes, s) == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+  }
+  CUtensorMap ma, mb;
+  if (!gemm::make_map(&ma, A->codes, M, K, gemm::BM) || !gemm::make_map(&mb, B->codes, N, K, gemm::BN))
+    return FP4_ERR_CUDA;
+  gemm::Params p{};
+  p.M = M; p.N = N; p.K = K;
+  p.sfa = A->scales_swz; p.sfb = B->scales_swz;
+  p.nkb = (K / (A->fmt == FP4_NVFP4 ? 16 : 32) + 3) / 4;
+  p.ta = A->tensor_scale; p.tb = B->tensor_scale;
+  p.D = D; p.mask = epi_mask; p.status = status_ptr();
+  cudaError_t e;
+  const bool nv = A->fmt == FP4_NVFP4, bf = out_dtype == 1, epi = epi_inverse_had == 32;
+  if (nv) {
+    if (bf) e = epi ? gemm::launch<1, 1, 1>(ma, mb, p, s) : gemm::launch<1, 1, 0>(ma, mb, p, s);
+    else e = epi ? gemm::launch<1, 0, 1>(ma, mb, p, s) : gemm::launch<1, 0, 0>(ma, mb, p, s);
+  } else {
+    if (bf) e = epi ? gemm::launch<0, 1, 1>(ma, mb, p, s) : gemm::launch<0, 1, 0>(ma, mb, p, s);
+    else e = epi ? gemm::launch<0, 0, 1>(ma, mb, p, s) : gemm::launch<0, 0, 0>(ma, mb, p, s);
+  }
+  return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}

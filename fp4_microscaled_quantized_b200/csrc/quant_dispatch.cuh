@@ -1,0 +1,70 @@
+// Host-side launch of the quantiser kernels for one loader (instantiated once
+// per loader in quant_ld*.cu so the four compile in parallel).
+#pragma once
+#include "quant_kernels.cuh"
+
+namespace fp4 {
+
+template <int LOAD>
+cudaError_t launch_quant(int fmt, int rnd, int had, const QParams& p, cudaStream_t s);
+
+int num_sms();
+
+template <int LOAD, int FMT, int RND, int HAD>
+cudaError_t launch_one(const QParams& p, cudaStream_t s) {
+  if (LOAD == LD_ROW || LOAD == LD_ROW_FP4) {
+    int64_t tasks = p.rows * (p.cols >> 3);
+    int64_t blocks = (tasks + 255) / 256;
+    int64_t cap = int64_t(num_sms()) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    k_quant_row<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
+  } else {
+    dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
+              unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
+    k_quant_trans<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+#define FP4_HAD_SWITCH(LOAD, FMT, RND)                                      \
+  switch (had) {                                                            \
+    case 0: return launch_one<LOAD, FMT, RND, 0>(p, s);                     \
+    case 16: return launch_one<LOAD, FMT, RND, 16>(p, s);                   \
+    case 32: return launch_one<LOAD, FMT, RND, 32>(p, s);                   \
+    case 128: return launch_one<LOAD, FMT, RND, 128>(p, s);                 \
+    default: return cudaErrorInvalidValue;                                  \
+  }
+
+#define FP4_HAD_SWITCH_ROT(LOAD, FMT, RND)                                  \
+  switch (had) {                                                            \
+    case 16: return launch_one<LOAD, FMT, RND, 16>(p, s);                   \
+    case 32: return launch_one<LOAD, FMT, RND, 32>(p, s);                   \
+    case 128: return launch_one<LOAD, FMT, RND, 128>(p, s);                 \
+    default: return cudaErrorInvalidValue;                                  \
+  }
+
+#define FP4_DEFINE_LAUNCH_QUANT(LOAD)                                               \
+  template <>                                                                       \
+  cudaError_t launch_quant<LOAD>(int fmt, int rnd, int had, const QParams& p,       \
+                                 cudaStream_t s) {                                  \
+    if (rnd == R_AMAX) { FP4_HAD_SWITCH(LOAD, FMT_NV, R_AMAX) }                     \
+    if (fmt == FMT_NV) {                                                            \
+      switch (rnd) {                                                                \
+        case R_RTN: { FP4_HAD_SWITCH(LOAD, FMT_NV, R_RTN) }                         \
+        case R_QUEST: { FP4_HAD_SWITCH(LOAD, FMT_NV, R_QUEST) }                     \
+        case R_FOS: { FP4_HAD_SWITCH(LOAD, FMT_NV, R_FOS) }                         \
+        case R_SR: { FP4_HAD_SWITCH(LOAD, FMT_NV, R_SR) }                           \
+        case R_EDEN: { FP4_HAD_SWITCH_ROT(LOAD, FMT_NV, R_EDEN) }                   \
+        default: return cudaErrorInvalidValue;                                      \
+      }                                                                             \
+    }                                                                               \
+    switch (rnd) {                                                                  \
+      case R_RTN: { FP4_HAD_SWITCH(LOAD, FMT_MX, R_RTN) }                           \
+      case R_QUEST: { FP4_HAD_SWITCH(LOAD, FMT_MX, R_QUEST) }                       \
+      case R_SR: { FP4_HAD_SWITCH(LOAD, FMT_MX, R_SR) }                             \
+      default: return cudaErrorInvalidValue;                                        \
+    }                                                                               \
+  }
+
+}  // namespace fp4

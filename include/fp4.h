@@ -1,0 +1,155 @@
+/*
+ * fp4.h -- C ABI of the B200 (sm_100a) fully-FP4 linear layer.
+ *
+ * The method follows three pages:
+ *  [Q]   "Quartet: Native FP4 Training Can Be Optimal for Large Language
+ *        Models" -- MXFP4 training (Hadamard-32 + QuEST forward, randomized
+ *        Hadamard + SR(3/4) backward, clip-mask epilogue), Algorithm 1;
+ *  [QII] "Quartet II: Accurate LLM Pre-Training in NVFP4 by Improved
+ *        Unbiased Gradient Estimation" -- NVFP4 format and NVIDIA-style SR,
+ *        Four-Over-Six, MS-EDEN (Algorithm 1) and its post hoc range
+ *        alignment, the Quartet II computation graph;
+ *  [BG]  "Bridging the Gap Between Promise and Performance for Microscaling
+ *        FP4 Quantization" -- MXFP4 / NVFP4 formats.
+ *
+ * Conventions for every call
+ *  - All pointers named *_dev, and every pointer inside fp4_qtensor, are
+ *    DEVICE pointers owned by the caller; the library allocates nothing and
+ *    keeps no reference after the call returns.  Host pointers (structs
+ *    passed by address) are read during the call only.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  The returned int is a synchronous fp4_status for
+ *    argument errors or launch failures.  Errors found on the device
+ *    (non-finite input, bounded-wait timeout) are recorded in a device
+ *    status word read (and cleared) by fp4_get_last_error().
+ *  - Matrices are row-major.  A quantised tensor of shape rows x cols has
+ *    its scale groups along cols (the GEMM's inner dimension).
+ *  - FP4 codes: E2M1, 2 per byte, element 2j in bits 0-3 and element 2j+1
+ *    in bits 4-7 of byte j of the row; code = sign << 3 | magnitude index of
+ *    {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *  - Linear scales: rows x (cols / g) bytes, row-major.  MXFP4: E8M0
+ *    (2^(c-127)), g = 32.  NVFP4: E4M3, g = 16, times the fp32 tensor scale.
+ *  - Swizzled scales (the tensor-core block-scale layout): 512-byte atoms
+ *    covering 128 rows x 4 groups; byte (r, k) lives at
+ *      ((r / 128) * nkb + k / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + k % 4
+ *    with nkb = ceil((cols / g) / 4); rows pad to 128 and groups to 4 with
+ *    zeros.  Size: ceil(rows / 128) * nkb * 512 bytes.
+ *  - QuEST clip mask: rows x (cols / 8) bytes, element 8b + j in bit j of
+ *    byte b; 1 = the element was clipped.
+ */
+#ifndef FP4_B200_H
+#define FP4_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *fp4_stream_t; /* == cudaStream_t */
+
+enum fp4_status {
+  FP4_OK = 0,
+  FP4_ERR_INVALID_ARG = 1,      /* null pointer, bad size, bad enum value   */
+  FP4_ERR_UNSUPPORTED = 2,      /* combination the pages do not define      */
+  FP4_ERR_ALIGNMENT = 3,        /* pointer or dimension alignment violated  */
+  FP4_ERR_WORKSPACE = 4,        /* workspace missing or too small           */
+  FP4_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed     */
+  FP4_ERR_NONFINITE_INPUT = 6,  /* device: NaN or Inf seen in an input      */
+  FP4_ERR_TIMEOUT = 7           /* device: a bounded wait gave up           */
+};
+
+enum fp4_format { FP4_MXFP4 = 0, FP4_NVFP4 = 1 };
+
+enum fp4_rounding {
+  FP4_RTN = 0,           /* AbsMax scale, round to nearest [Q]; [QII] Alg. 1 step 2 */
+  FP4_QUEST = 1,         /* RMSE-optimal clipping + clip mask [Q] "QuEST in Detail" */
+  FP4_FOUR_OVER_SIX = 2, /* NVFP4 only [QII] "Forward Pass Design"                  */
+  FP4_SR = 3,            /* NVFP4: [QII] standard SR steps 1-3; MXFP4: SR(3/4 x) [Q] */
+  FP4_MS_EDEN = 4        /* NVFP4 only, needs a rotation [QII] MS-EDEN, post hoc     */
+};
+
+/* Block Hadamard along the inner dimension [Q] "The Hadamard Transform".
+ * block: 0 (none), 16, 32 or 128.  randomized: 0 = H_g, 1 = H_g diag(d)
+ * with d_j = +-1 drawn from Philox(seed, counter (j/4, 0, 3, sign_tag)), one
+ * pattern for every block of the tensor; two operands of one GEMM must use
+ * the same seed and sign_tag so the rotations cancel [QII] MS-EDEN step 1. */
+typedef struct {
+  int32_t block;
+  int32_t randomized;
+  uint32_t sign_tag;
+} fp4_had;
+
+typedef struct {
+  uint8_t *codes;      /* rows x cols/2, required                              */
+  uint8_t *scales;     /* rows x cols/g linear; may be NULL if scales_swz set  */
+  uint8_t *scales_swz; /* tensor-core layout; may be NULL if scales set        */
+  float *tensor_scale; /* 1 float: NVFP4 fp32 scale; MXFP4 1.0 (4/3 for SR)    */
+  uint8_t *mask;       /* rows x cols/8, QuEST only (else NULL)                */
+  int64_t rows;        /* shape of the QUANTISED tensor                        */
+  int64_t cols;
+  int32_t fmt;         /* fp4_format                                           */
+  int32_t reserved;
+} fp4_qtensor;
+
+/* Bytes of device workspace fp4_quantize / fp4_requantize need for a
+ * quantised tensor of rows x cols (16-byte multiple; 0 for modes without a
+ * global pass).  NVFP4 RTN/QuEST/4-6/SR: one amax word.  MS-EDEN: amax, the
+ * bf16 E8M3 pseudo-scales (rows * cols/16 * 2) and the fp32 EDEN factors
+ * (rows * cols/block * 4) of the post hoc range alignment [QII]. */
+size_t fp4_quantize_workspace_size(int64_t rows, int64_t cols, int32_t fmt,
+                                   int32_t rounding, int32_t had_block);
+
+/* Bytes of the swizzled scale buffer for rows x n_groups scales. */
+size_t fp4_swizzled_scale_bytes(int64_t rows, int64_t n_groups);
+
+/* y = block (randomized) Hadamard of x along cols, fp32 out.
+ * x_dev: rows x cols bf16; y_dev: rows x cols fp32; cols % block == 0.
+ * [Q] "The Hadamard Transform": Sylvester order, 1/sqrt(g) normalisation. */
+int fp4_hadamard(const void *x_dev, float *y_dev, int64_t rows, int64_t cols,
+                 fp4_had had, uint64_t seed, fp4_stream_t stream);
+
+/* Quantise a bf16 matrix.  x_dev is in_rows x in_cols; with transpose = 0 the
+ * quantised tensor is x (rows = in_rows, cols = in_cols), with transpose = 1
+ * it is x^T (rows = in_cols, cols = in_rows), i.e. the groups and the
+ * rotation run along x's rows -- the backward operands of [QII] "The
+ * Complete Quartet II Computation Graph".  group must equal the format's
+ * group size (16 NVFP4, 32 MXFP4).  cols must be a multiple of
+ * max(group, had.block); with transpose = 1, in_cols must be a multiple of 8.
+ * seed/tensor_tag key the Philox streams of SR (element index in the output
+ * layout) and MS-EDEN (group index).  out: caller fills the pointers; the
+ * call writes rows, cols and fmt.  ws_dev: fp4_quantize_workspace_size bytes,
+ * 16-byte aligned, contents need not be initialised. */
+int fp4_quantize(const void *x_dev, int64_t in_rows, int64_t in_cols,
+                 int32_t transpose, int32_t fmt, int32_t rounding, int32_t group,
+                 fp4_had had, uint64_t seed, uint32_t tensor_tag,
+                 fp4_qtensor *out, void *ws_dev, size_t ws_bytes,
+                 fp4_stream_t stream);
+
+/* Re-quantise a saved FP4 tensor [QII] computation graph backward steps 1-4:
+ * de-quantise (fp32(fp32(q * s_group) * s_tensor)), optionally transpose,
+ * rotate along the new inner dimension, quantise in `in->fmt` with
+ * `rounding`.  in->scales (linear) is required. */
+int fp4_requantize(const fp4_qtensor *in, int32_t transpose, int32_t rounding,
+                   fp4_had had, uint64_t seed, uint32_t tensor_tag,
+                   fp4_qtensor *out, void *ws_dev, size_t ws_bytes,
+                   fp4_stream_t stream);
+
+/* Linear (rows x n_groups) scales -> the swizzled tensor-core layout
+ * (padding zeroed).  [Q] "Stage 2", scale factor layout. */
+int fp4_swizzle_scales(const uint8_t *scales_dev, int64_t rows, int64_t n_groups,
+                       uint8_t *scales_swz_dev, fp4_stream_t stream);
+
+/* Read and clear the device status word after synchronising `stream`.
+ * Returns FP4_OK or the first device-side fp4_status recorded. */
+int fp4_get_last_error(fp4_stream_t stream);
+
+/* Static description of a status code. */
+const char *fp4_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4_B200_H */

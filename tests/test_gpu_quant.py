@@ -1,0 +1,125 @@
+"""GPU parity of the Hadamard / quantise / pack / swizzle kernels against the
+oracle: bit-exact codes, scale bytes, tensor-scale bits and mask bits in
+every mode (the stochastic ones draw the same Philox bits)."""
+import numpy as np
+import pytest
+import torch
+
+from fp4_microscaled_quantized_b200 import synthetic as syn
+from oracle import formats as fm
+from oracle import hadamard as hd
+from oracle import quant as qn
+
+pytestmark = pytest.mark.gpu
+
+COMBOS = [(f, r, h) for f in (qn.MXFP4, qn.NVFP4) for r in range(5) for h in (0, 16, 32, 128)
+          if qn.supported(f, r, h)]
+
+
+def to_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def assert_qt_equal(g, o, check_mask=True):
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(g.codes.cpu().numpy(), fm.pack_codes(o.codes), err_msg="codes")
+    np.testing.assert_array_equal(g.scales.cpu().numpy(), o.scales, err_msg="scales")
+    swz = g.scales_swz.cpu().numpy()
+    np.testing.assert_array_equal(swz, qn.swizzle_scales(o.scales), err_msg="swizzled scales")
+    assert g.tensor_scale.cpu().numpy().view(np.uint32)[0] == np.float32(o.tensor_scale).view(np.uint32)
+    if check_mask and o.mask is not None:
+        np.testing.assert_array_equal(g.mask.cpu().numpy(), fm.pack_mask(o.mask), err_msg="mask")
+
+
+@pytest.mark.parametrize("fmt,rnd,had", COMBOS)
+@pytest.mark.parametrize("transpose", [False, True])
+def test_quantize_parity(cuda_lib, fmt, rnd, had, transpose):
+    shape = (512, 200) if transpose else (200, 512)
+    bits = syn.outlier_elements(shape, seed=7, stream=fmt * 10 + rnd)
+    x = syn.bf16_bits_to_f32(bits)
+    seed, stag, ttag = 0x1234ABCD5678, 1, 9
+    g = cuda_lib.quantize(to_dev(bits), fmt, rnd, had, randomized=had > 0, seed=seed,
+                          sign_tag=stag, tensor_tag=ttag, transpose=transpose)
+    o = qn.quantize(x, fmt, rnd, had, had > 0, seed, stag, ttag, transpose=transpose)
+    assert_qt_equal(g, o)
+    assert cuda_lib.get_last_error() == 0
+
+
+@pytest.mark.parametrize("fmt,fwd_rnd,rnd,had", [
+    (qn.NVFP4, qn.FOUR_OVER_SIX, qn.MS_EDEN, 128), (qn.NVFP4, qn.FOUR_OVER_SIX, qn.SR, 16),
+    (qn.NVFP4, qn.RTN, qn.RTN, 0), (qn.MXFP4, qn.QUEST, qn.SR, 32), (qn.MXFP4, qn.RTN, qn.QUEST, 32)])
+@pytest.mark.parametrize("transpose", [True, False])
+def test_requantize_parity(cuda_lib, fmt, fwd_rnd, rnd, had, transpose):
+    """De-quantise a saved (oracle-quantised) tensor, transpose, rotate,
+    quantise again (Quartet II computation graph, backward steps 1-4)."""
+    bits = syn.student_t((384, 256), seed=3, unit_rms=True)
+    x = syn.bf16_bits_to_f32(bits)
+    saved = qn.quantize(x, fmt, fwd_rnd, 0)
+    dev = cuda_lib.alloc_qtensor(384, 256, fmt, mask=False)
+    dev.codes.copy_(torch.from_numpy(fm.pack_codes(saved.codes)))
+    dev.scales.copy_(torch.from_numpy(saved.scales))
+    dev.tensor_scale.copy_(torch.tensor([float(saved.tensor_scale)], dtype=torch.float32))
+    seed = 77
+    g = cuda_lib.requantize(dev, rnd, had, randomized=had > 0, seed=seed, sign_tag=2, tensor_tag=4,
+                            transpose=transpose)
+    o = qn.requantize(saved, rnd, had, had > 0, seed, 2, 4, transpose=transpose)
+    assert_qt_equal(g, o)
+
+
+@pytest.mark.parametrize("block", [16, 32, 128])
+@pytest.mark.parametrize("randomized", [False, True])
+def test_hadamard_parity(cuda_lib, block, randomized):
+    bits = syn.gaussian((96, 512), 1.0, seed=5)
+    y = cuda_lib.hadamard(to_dev(bits), block, randomized, seed=42, sign_tag=3)
+    o = hd.block_transform(syn.bf16_bits_to_f32(bits), block, randomized, 42, 3)
+    np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), o.view(np.uint32))
+
+
+def test_swizzle_kernel(cuda_lib):
+    s = np.random.default_rng(0).integers(0, 255, (300, 10)).astype(np.uint8)
+    out = cuda_lib.swizzle_scales(torch.from_numpy(s).cuda())
+    np.testing.assert_array_equal(out.cpu().numpy(), qn.swizzle_scales(s))
+
+
+def test_multi_tile_large_parity(cuda_lib):
+    """Several row tiles, a ragged row count and a 4096-wide inner dimension
+    through the grid-stride loop (config-5 row length)."""
+    bits = syn.quantizer_sweep(4096 * 1000 + 4096 * 37, seed=7)
+    x = syn.bf16_bits_to_f32(bits)
+    for fmt, rnd, had in [(qn.NVFP4, qn.MS_EDEN, 128), (qn.NVFP4, qn.FOUR_OVER_SIX, 0),
+                          (qn.MXFP4, qn.SR, 32)]:
+        g = cuda_lib.quantize(to_dev(bits), fmt, rnd, had, randomized=True, seed=5, sign_tag=0,
+                              tensor_tag=1)
+        o = qn.quantize(x, fmt, rnd, had, True, 5, 0, 1)
+        assert_qt_equal(g, o)
+
+
+def test_nonfinite_input_flags_status(cuda_lib):
+    bits = syn.gaussian((64, 256), 1.0, seed=1)
+    bits[3, 17] = 0x7FC0                                   # NaN
+    for fmt, rnd, had in [(qn.NVFP4, qn.RTN, 0), (qn.NVFP4, qn.MS_EDEN, 128), (qn.MXFP4, qn.QUEST, 32)]:
+        cuda_lib.quantize(to_dev(bits), fmt, rnd, had, randomized=True)
+        assert cuda_lib.get_last_error() == 6
+        assert cuda_lib.get_last_error() == 0              # cleared by the read
+
+
+def test_argument_errors(cuda_lib):
+    x = to_dev(syn.gaussian((64, 256), 1.0, seed=1))
+    with pytest.raises(cuda_lib.Fp4Error) as e:
+        cuda_lib.quantize(x, qn.MXFP4, qn.MS_EDEN, 128)
+    assert e.value.status == 2
+    with pytest.raises(cuda_lib.Fp4Error) as e:
+        cuda_lib.quantize(x, qn.NVFP4, qn.MS_EDEN, 0)
+    assert e.value.status == 2
+    with pytest.raises(cuda_lib.Fp4Error) as e:
+        cuda_lib.quantize(to_dev(syn.gaussian((64, 200), 1.0, 1)), qn.NVFP4, qn.RTN, 128)
+    assert e.value.status == 1                             # 200 % 128 != 0
+    with pytest.raises(cuda_lib.Fp4Error) as e:
+        cuda_lib.quantize(x, qn.NVFP4, qn.MS_EDEN, 128, ws=cuda_lib.alloc_workspace(16))
+    assert e.value.status == 4
+
+
+def test_empty_input_is_a_noop(cuda_lib):
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    q = cuda_lib.quantize(x, qn.NVFP4, qn.MS_EDEN, 128)
+    assert q.rows == 0 and cuda_lib.get_last_error() == 0
