@@ -83,8 +83,7 @@ def _declare_extra(lib):
     P, I32, I64, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
     QP = ctypes.POINTER(fp4_qtensor)
     extra = {
-        "fp4_gemm": (ctypes.c_int, [QP, QP, P, I32, P, I32, P, SZ, P]),
-        "fp4_gemm_workspace_size": (SZ, [I64, I64, I64]),
+        "fp4_gemm": (ctypes.c_int, [QP, QP, P, I32, P, I32, P]),
     }
     for name, (res, args) in extra.items():
         if hasattr(lib, name):
@@ -204,6 +203,19 @@ def swizzle_scales(scales):
     out = torch.empty((max(lib.fp4_swizzled_scale_bytes(rows, ng), 1),), dtype=torch.uint8,
                       device=scales.device)
     _check(lib.fp4_swizzle_scales(_ptr(scales), rows, ng, _ptr(out), _stream()), "fp4_swizzle_scales")
+    return out
+
+
+def gemm(A, B, out_dtype=torch.float32, mask=None, inverse_had=0, out=None):
+    """fp4_gemm: D = dq(A) dq(B)^T (optionally the Quartet mask + H32^-1 epilogue)."""
+    lib = load()
+    if out is None:
+        out = torch.empty((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
+    code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
+    ca, cb = A.c_struct(), B.c_struct()
+    st = lib.fp4_gemm(ctypes.byref(ca), ctypes.byref(cb), _ptr(out), code, _ptr(mask),
+                      inverse_had, _stream())
+    _check(st, "fp4_gemm")
     return out
 
 

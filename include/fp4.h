@@ -141,6 +141,21 @@ int fp4_requantize(const fp4_qtensor *in, int32_t transpose, int32_t rounding,
 int fp4_swizzle_scales(const uint8_t *scales_dev, int64_t rows, int64_t n_groups,
                        uint8_t *scales_swz_dev, fp4_stream_t stream);
 
+/* Block-scaled FP4 GEMM on the tcgen05 tensor cores [Q] "Stage 2":
+ *   D = (A . SFA) (B . SFB)^T * (tA * tB)
+ * A: M x K quantised tensor (A->rows = M, A->cols = K), B: N x K (B->rows = N),
+ * same format; both K-major with swizzled scales (scales_swz required).
+ * D_dev: M x N row-major, fp32 (out_dtype 0) or bf16 (out_dtype 1, rounded
+ * to nearest even), FP32 accumulation.  K % 64 == 0, N % 8 == 0.
+ * epi_inverse_had = 32 applies the Quartet backward epilogue
+ * [Q] "Inverse Hadamard and clipping mask correction": every 32-column block
+ * of the scaled product is multiplied by (1 - mask) (mask: M x N/8 bytes,
+ * 1 = clipped in the forward pass; NULL = no mask) and then by H32^-1 = H32;
+ * requires N % 32 == 0.  The 16/9 factor is the product of the operands'
+ * tensor scales (4/3 each).  epi_inverse_had = 0 and a mask is an error. */
+int fp4_gemm(const fp4_qtensor *A, const fp4_qtensor *B, void *D_dev, int32_t out_dtype,
+             const uint8_t *epi_mask_dev, int32_t epi_inverse_had, fp4_stream_t stream);
+
 /* Read and clear the device status word after synchronising `stream`.
  * Returns FP4_OK or the first device-side fp4_status recorded. */
 int fp4_get_last_error(fp4_stream_t stream);
