@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the fully-FP4 linear layer on B200.
+
+Workload: the Llama-3-8B-shaped layer set in the Quartet II NVFP4 recipe,
+M = 16384 tokens, layers QKV 4096->6144, O 4096->4096, gate/up 4096->28672
+(2 x 14336 as one GEMM), down 14336->4096.  One step = forward + backward of
+all four layers: Four-Over-Six quantisation of X and W, the forward GEMM,
+MS-EDEN (RHT-128) quantisation of dY row-wise and transposed, re-quantisation
+of the saved Q(W)^T and Q(X)^T, and the dX and dW GEMMs, all through the C ABI.
+Metric: end-to-end TFLOP/s = 6 M sum(N K) / step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (one per rank, launched by torchrun); the
+step time is the max over ranks.  Prints one JSON line on rank 0.
+"""
+import argparse
+import ctypes
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from fp4_microscaled_quantized_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "NVFP4 linear fwd+bwd TFLOPS and quantizer HBM GB/s vs roofline, 1xB200"
+UNIT = "TFLOP/s"
+M_TOKENS = 16384
+LAYERS = syn.LLAMA3_8B_LAYERS          # (name, K = in_features, N = out_features)
+TAG_E_ROW, TAG_W_T, TAG_E_T, TAG_X_T, TAG_X, TAG_W = 1, 2, 3, 4, 5, 6
+GEMM_DX, GEMM_DW = 0, 1
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0                    # nominal dense ratio 9 / 2.25 PFLOP/s
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=M_TOKENS)
+    ap.add_argument("--layers", default="qkv,o,gate_up,down",
+                    help="subset of the layer set (profiling small cases)")
+    args = ap.parse_args()
+    global LAYERS
+    keep = args.layers.split(",")
+    LAYERS = tuple(L for L in syn.LLAMA3_8B_LAYERS if L[0] in keep)
+    return args
+
+
+# --------------------------------------------------------------- ranks --
+def init_dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    """Max of a float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------- clocks --
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            sel = str(self.dev)
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in rows if num(r[0]) is not None]
+        pw = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i].lower().startswith("active")})
+        loaded = [s for s, p in zip(sm, pw) if p is not None and p > 300] or sm
+        return {"sm_mhz": float(np.median(loaded)) if loaded else None,
+                "sm_max_mhz": num(rows[0][1]), "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(pw) if pw else None}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------ workload --
+def make_host_data(M):
+    """Seeded synthetic bf16 inputs of every layer (Quartet II distributions),
+    in pinned host memory."""
+    out = []
+    for li, (name, K, N) in enumerate(LAYERS):
+        d = syn.linear_quartet2(M, N, K, 3 + li)
+        out.append({k: torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).pin_memory()
+                    for k, v in d.items()})
+    return out
+
+
+def quant_bytes_per_elem(kind):
+    """Algorithmic HBM bytes per quantised element of each quantiser call
+    (bf16 read 2 B; codes 0.5; one scale copy 1/16; MS-EDEN pseudo-scales
+    bf16 written and read back 2 x 2/16; EDEN factors 2 x 4/128)."""
+    if kind == "fos":            # amax pass + quantise pass over bf16
+        return 2 + 2 + 0.5 + 1 / 16
+    if kind == "eden":           # post hoc: one bf16 read, scales-only second pass
+        return 2 + 0.5 + 1 / 16 + 2 * 2 / 16 + 2 * 4 / 128
+    if kind == "eden_requant":   # saved FP4 (codes + scales) in, FP4 out
+        return 0.5 + 1 / 16 + 0.5 + 1 / 16 + 2 * 2 / 16 + 2 * 4 / 128
+    raise ValueError(kind)
+
+
+class Step:
+    """One fwd+bwd pass over the layer set through the C ABI's quantise /
+    re-quantise / GEMM entry points (the same kernel sequence fp4_linear_fwd
+    and fp4_linear_bwd issue), with CUDA events around every call."""
+
+    def __init__(self, api, M, device, host):
+        self.api = api
+        self.M = M
+        self.r = api.recipe(api.RECIPE_QUARTET2)
+        self.layers = []
+        for li, (name, K, N) in enumerate(LAYERS):
+            d = {k: v.to(device) for k, v in host[li].items()}
+            L = {"name": name, "K": K, "N": N, **d}
+            L["ctx"] = api.alloc_ctx(self.r, M, N, K, device)
+            L["Y"] = torch.empty((M, N), dtype=torch.float32, device=device)
+            L["dX"] = torch.empty((M, K), dtype=torch.float32, device=device)
+            L["dW"] = torch.empty((N, K), dtype=torch.float32, device=device)
+            L["e_row"] = api.alloc_qtensor(M, N, api.NVFP4, linear=False)
+            L["w_t"] = api.alloc_qtensor(K, N, api.NVFP4, linear=False)
+            L["e_t"] = api.alloc_qtensor(N, M, api.NVFP4, linear=False)
+            L["x_t"] = api.alloc_qtensor(K, M, api.NVFP4, linear=False)
+            self.layers.append(L)
+        need = max(api.workspace_size(a, b, api.NVFP4, api.MS_EDEN, 128)
+                   for L in self.layers for a, b in ((M, L["N"]), (L["K"], L["N"]), (L["N"], M), (L["K"], M)))
+        self.ws = api.alloc_workspace(need, device)
+        self.records = []
+        self.flops = sum(6.0 * M * L["N"] * L["K"] for L in self.layers)
+
+    def _ev(self, kind, elems, fn):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        self.records.append((kind, elems, a, b))
+
+    def run(self, step_seed, record=True):
+        api, M, ws = self.api, self.M, self.ws
+        ev = self._ev if record else (lambda kind, elems, fn: fn())
+        for L in self.layers:
+            K, N, ctx = L["K"], L["N"], L["ctx"]
+            ev("fos", M * K, lambda: api.quantize(L["X"], api.NVFP4, api.FOUR_OVER_SIX, 0, tensor_tag=TAG_X,
+                                                  out=ctx.xq, ws=ws))
+            ev("fos", N * K, lambda: api.quantize(L["W"], api.NVFP4, api.FOUR_OVER_SIX, 0, tensor_tag=TAG_W,
+                                                  out=ctx.wq, ws=ws))
+            ev("gemm", 2.0 * M * N * K, lambda: api.gemm(ctx.xq, ctx.wq, out=L["Y"]))
+            ev("eden", M * N, lambda: api.quantize(L["dY"], api.NVFP4, api.MS_EDEN, 128, True, step_seed,
+                                                   GEMM_DX, TAG_E_ROW, out=L["e_row"], ws=ws))
+            ev("eden_requant", N * K, lambda: api.requantize(ctx.wq, api.MS_EDEN, 128, True, step_seed, GEMM_DX,
+                                                             TAG_W_T, transpose=True, out=L["w_t"], ws=ws))
+            ev("gemm", 2.0 * M * N * K, lambda: api.gemm(L["e_row"], L["w_t"], out=L["dX"]))
+            ev("eden", M * N, lambda: api.quantize(L["dY"], api.NVFP4, api.MS_EDEN, 128, True, step_seed,
+                                                   GEMM_DW, TAG_E_T, transpose=True, out=L["e_t"], ws=ws))
+            ev("eden_requant", M * K, lambda: api.requantize(ctx.xq, api.MS_EDEN, 128, True, step_seed, GEMM_DW,
+                                                             TAG_X_T, transpose=True, out=L["x_t"], ws=ws))
+            ev("gemm", 2.0 * M * N * K, lambda: api.gemm(L["e_t"], L["x_t"], out=L["dW"]))
+
+    def summary(self):
+        g_t = g_f = q_t = q_b = 0.0
+        n_gemm = 0
+        for kind, elems, a, b in self.records:
+            ms = a.elapsed_time(b)
+            if kind == "gemm":
+                g_t += ms
+                g_f += elems
+                n_gemm += 1
+            else:
+                q_t += ms
+                q_b += elems * quant_bytes_per_elem(kind)
+        return {"gemm_ms": g_t, "gemm_flops": g_f, "n_gemm": n_gemm, "quant_ms": q_t, "quant_bytes": q_b}
+
+
+def run_e2e(api, M, steps, device, host):
+    """Same metric through the public linear-layer API with host buffers:
+    every step copies X, W, dY of every layer host->device (pinned), runs
+    fp4_linear_fwd + fp4_linear_bwd and reads dW back device->host."""
+    r = api.recipe(api.RECIPE_QUARTET2)
+    devbuf = []
+    for li, (name, K, N) in enumerate(LAYERS):
+        d = host[li]
+        devbuf.append({"X": torch.empty_like(d["X"], device=device), "W": torch.empty_like(d["W"], device=device),
+                       "dY": torch.empty_like(d["dY"], device=device),
+                       "ctx": api.alloc_ctx(r, M, N, K, device),
+                       "Y": torch.empty((M, N), dtype=torch.float32, device=device),
+                       "dX": torch.empty((M, K), dtype=torch.float32, device=device),
+                       "dW": torch.empty((N, K), dtype=torch.float32, device=device),
+                       "dW_host": torch.empty((N, K), dtype=torch.float32).pin_memory(),
+                       "wsf": api.linear_workspace(r, M, N, K, False, device),
+                       "wsb": api.linear_workspace(r, M, N, K, True, device)})
+    h2d = sum(v.numel() * v.element_size() for h in host for v in h.values())
+    d2h = sum(b["dW"].numel() * 4 for b in devbuf)
+
+    def step(seed):
+        for h, b in zip(host, devbuf):
+            for k in ("X", "W", "dY"):
+                b[k].copy_(h[k], non_blocking=True)
+            api.linear_fwd(b["X"], b["W"], r, 0, ctx=b["ctx"], Y=b["Y"], ws=b["wsf"])
+            api.linear_bwd(b["dY"], b["ctx"], seed, dX=b["dX"], dW=b["dW"], ws=b["wsb"])
+            b["dW_host"].copy_(b["dW"], non_blocking=True)
+
+    step(0)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for k in range(steps):
+        step(100 + k)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    flops = sum(6.0 * M * N * K for _, K, N in LAYERS)
+    del devbuf
+    torch.cuda.empty_cache()
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
+
+
+# --------------------------------------------------------- CPU oracle --
+def oracle_sample(n_rows, n_out, seed=0):
+    """The oracle's fwd+bwd on a bounded sample of the same workload: the
+    first n_rows tokens and n_out output features of the QKV layer (full
+    K = 4096).  Single-threaded numpy (BLAS limited to one thread)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import linear as ln
+    K = LAYERS[0][1]
+    d = syn.linear_quartet2(n_rows, n_out, K, 3 + seed)
+    f = syn.bf16_bits_to_f32
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        _, _, ctx = ln.linear_fwd(f(d["X"]), f(d["W"]), ln.QUARTET2)
+        ln.linear_bwd(f(d["dY"]), ctx, ln.QUARTET2, 7)
+        dt = time.perf_counter() - t0
+    flops = 6.0 * n_rows * n_out * K
+    return flops, dt
+
+
+def cpu_baseline(target_s=15.0):
+    # calibrate on a small sample, then run one sized for about target_s
+    f0, t0 = oracle_sample(128, 256)
+    n_out = int(min(6144, max(256, 256 * target_s / max(t0, 1e-3))) // 128 * 128)
+    f1, t1 = oracle_sample(128, n_out)
+    return {"value": f1 / t1 / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "QKV layer, 128 tokens x %d output features x K=4096, Quartet II fwd+bwd "
+                      "(quantisers + fp64 GEMMs), %.1f s" % (n_out, t1)}
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return
+    per_step = max(3.0, 150.0 / max(1, args.steps + args.warmup))
+    f0, t0 = oracle_sample(128, 256)
+    n_out = int(min(6144, max(128, 256 * per_step / max(t0, 1e-3))) // 128 * 128)
+    for _ in range(args.warmup):
+        oracle_sample(128, n_out)
+    tot_f = tot_t = 0.0
+    for k in range(args.steps):
+        f, t = oracle_sample(128, n_out, seed=k)
+        tot_f += f
+        tot_t += t
+    v = tot_f / tot_t / 1e12
+    sample = "QKV layer, 128 tokens x %d output features x K=4096 per step, Quartet II fwd+bwd" % n_out
+    print(json.dumps({
+        "metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantisers, f64 GEMM",
+        "data": "synthetic", "config": config_dict(M_TOKENS),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+
+
+def config_dict(M):
+    return {"workload": "llama3-8b layer set (qkv 4096->6144, o 4096->4096, gate_up 4096->28672, "
+                        "down 14336->4096), NVFP4 Quartet II fwd+bwd",
+            "tokens": M, "recipe": "quartet2: RTN+4/6 fwd, RHT128 + MS-EDEN bwd", "outputs": "fp32 Y, dX, dW",
+            "global_batch": M, "l2": "inputs larger than L2 (about 9 GB touched per step)",
+            "parallelism": "replicas"}
+
+
+# ------------------------------------------------------------------ main --
+def main():
+    args = parse()
+    world, rank, local = init_dist()
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+    from fp4_microscaled_quantized_b200 import api
+    api.load()
+    dev = torch.device("cuda", local)
+    M = args.tokens
+    t_gen = time.perf_counter()
+    host = make_host_data(M)
+    t_gen = time.perf_counter() - t_gen
+    step = Step(api, M, dev, host)
+    for w in range(max(args.warmup, 3)):
+        step.run(1000 + w, record=False)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    lc0 = api.load().fp4_launch_count()
+    step.records = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for k in range(args.steps):
+        step.run(k)
+    end.record()
+    torch.cuda.synchronize()
+    lc1 = api.load().fp4_launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    st = step.summary()
+    err = api.get_last_error()
+    value = world * step.flops / (ms_max * 1e-3) / 1e12
+
+    peaks, src = load_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    g_ach = st["gemm_flops"] / (st["gemm_ms"] * 1e-3) / 1e12
+    q_ach = st["quant_bytes"] / (st["quant_ms"] * 1e-3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(tpath):
+        traffic = json.load(open(tpath)).get("bytes_per_launch")
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, e4m3 scales, fp32 accumulate)",
+        "data": "synthetic (seeded Student-t / Gaussian, Quartet II distributions)",
+        "config": config_dict(M),
+        "roofline": {"bound": "tensor", "achieved": g_ach, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": g_ach / fp4_peak, "traffic": traffic,
+                     "kernel": "k_gemm (tcgen05 mxf4nvf4)",
+                     "peak_source": "%s cuBLAS bf16 sustained %.1f x %.0f (nominal fp4/bf16)" % (
+                         src, peaks["bf16_tflops_sustained"], FP4_OVER_BF16)},
+        "quantizers": {"achieved": q_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": q_ach / peaks["hbm_gbs"], "share_of_step": st["quant_ms"] / (ms * args.steps),
+                       "peak_source": src + " copy bandwidth"},
+        "gemm_share_of_step": st["gemm_ms"] / (ms * args.steps),
+        "clocks": clk, "gpu_launches": int(lc1 - lc0), "device_status": err,
+        "input_generation_s": round(t_gen, 1),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline()
+    del step
+    torch.cuda.empty_cache()
+    if args.e2e_steps > 0:
+        e2e = run_e2e(api, M, args.e2e_steps, dev, host)
+        e2e["value"] = world * e2e["value"] * (e2e["ms_per_step"] / max_over_ranks(e2e["ms_per_step"], world))
+        out["e2e"] = e2e
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

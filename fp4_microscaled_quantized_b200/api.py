@@ -82,8 +82,14 @@ def _declare_extra(lib):
     """Entry points added by later layers (GEMM, linear)."""
     P, I32, I64, U64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
     QP = ctypes.POINTER(fp4_qtensor)
+    RP = ctypes.POINTER(fp4_recipe)
+    CP = ctypes.POINTER(fp4_ctx)
     extra = {
         "fp4_gemm": (ctypes.c_int, [QP, QP, P, I32, P, I32, P]),
+        "fp4_recipe_preset": (ctypes.c_int, [I32, RP]),
+        "fp4_linear_workspace_size": (SZ, [RP, I64, I64, I64, I32]),
+        "fp4_linear_fwd": (ctypes.c_int, [P, P, I64, I64, I64, RP, U64, P, CP, P, SZ, P]),
+        "fp4_linear_bwd": (ctypes.c_int, [P, CP, I64, I64, I64, RP, U64, P, P, P, SZ, P]),
     }
     for name, (res, args) in extra.items():
         if hasattr(lib, name):
@@ -217,6 +223,104 @@ def gemm(A, B, out_dtype=torch.float32, mask=None, inverse_had=0, out=None):
                       inverse_had, _stream())
     _check(st, "fp4_gemm")
     return out
+
+
+RECIPE_QUARTET, RECIPE_QUARTET2, RECIPE_RTN = 0, 1, 2
+
+
+class fp4_recipe(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("fmt", "fwd_rounding", "fwd_had", "bwd_rounding", "bwd_had",
+                                               "bwd_randomized", "mask_epilogue", "out_y", "out_dx",
+                                               "out_dw")]
+
+
+class fp4_ctx(ctypes.Structure):
+    _fields_ = [("xq", fp4_qtensor), ("wq", fp4_qtensor)]
+
+
+def recipe(preset):
+    r = fp4_recipe()
+    _check(load().fp4_recipe_preset(preset, ctypes.byref(r)), "fp4_recipe_preset")
+    return r
+
+
+@dataclass
+class LinearCtx:
+    """Saved forward context: the quantised X (M x K) and W (N x K)."""
+    xq: QTensor
+    wq: QTensor
+    recipe: fp4_recipe
+
+    def c_struct(self):
+        return fp4_ctx(self.xq.c_struct(), self.wq.c_struct())
+
+
+_DT = {0: torch.float32, 1: torch.bfloat16}
+
+
+def linear_workspace(r, M, N, K, is_bwd, device="cuda"):
+    return alloc_workspace(load().fp4_linear_workspace_size(ctypes.byref(r), M, N, K, int(is_bwd)), device)
+
+
+def alloc_ctx(r, M, N, K, device="cuda"):
+    quest = r.fwd_rounding == QUEST
+    return LinearCtx(alloc_qtensor(M, K, r.fmt, mask=quest, device=device),
+                     alloc_qtensor(N, K, r.fmt, mask=quest, device=device), r)
+
+
+def linear_fwd(X, W, r, seed=0, ctx=None, Y=None, ws=None):
+    """fp4_linear_fwd: returns (Y, ctx)."""
+    lib = load()
+    M, K = X.shape
+    N = W.shape[0]
+    if ctx is None:
+        ctx = alloc_ctx(r, M, N, K, X.device)
+    if Y is None:
+        Y = torch.empty((M, N), dtype=_DT[r.out_y], device=X.device)
+    if ws is None:
+        ws = linear_workspace(r, M, N, K, False, X.device)
+    c = ctx.c_struct()
+    st = lib.fp4_linear_fwd(_ptr(X), _ptr(W), M, N, K, ctypes.byref(r), seed, _ptr(Y), ctypes.byref(c),
+                            _ptr(ws), ws.numel(), _stream())
+    _check(st, "fp4_linear_fwd")
+    return Y, ctx
+
+
+def linear_bwd(dY, ctx, step_seed, dX=None, dW=None, ws=None, want_dx=True, want_dw=True):
+    """fp4_linear_bwd: returns (dX, dW)."""
+    lib = load()
+    r = ctx.recipe
+    M, N = dY.shape
+    K = ctx.xq.cols
+    if want_dx and dX is None:
+        dX = torch.empty((M, K), dtype=_DT[r.out_dx], device=dY.device)
+    if want_dw and dW is None:
+        dW = torch.empty((N, K), dtype=_DT[r.out_dw], device=dY.device)
+    if ws is None:
+        ws = linear_workspace(r, M, N, K, True, dY.device)
+    c = ctx.c_struct()
+    st = lib.fp4_linear_bwd(_ptr(dY), ctypes.byref(c), M, N, K, ctypes.byref(r), step_seed,
+                            _ptr(dX if want_dx else None), _ptr(dW if want_dw else None),
+                            _ptr(ws), ws.numel(), _stream())
+    _check(st, "fp4_linear_bwd")
+    return dX, dW
+
+
+def selftest_e2m1():
+    """Mismatching 8-element words between the hardware E2M1 encoder and the
+    per-element rounding over all 2^32 fp32 patterns (0 expected)."""
+    lib = load()
+    lib.fp4_selftest_e2m1.restype = ctypes.c_int
+    lib.fp4_selftest_e2m1.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    cnt = torch.zeros((1,), dtype=torch.int64, device="cuda")
+    _check(lib.fp4_selftest_e2m1(_ptr(cnt), _stream()), "fp4_selftest_e2m1")
+    return int(cnt.item())
+
+
+def launch_count():
+    lib = load()
+    lib.fp4_launch_count.restype = ctypes.c_ulonglong
+    return int(lib.fp4_launch_count())
 
 
 def get_last_error():

@@ -1,5 +1,6 @@
 // C ABI entry points of the quantisation path (include/fp4.h): argument
 // validation, workspace layout, kernel sequencing and the device status word.
+#include <atomic>
 #include <mutex>
 
 #include "../../include/fp4.h"
@@ -8,6 +9,9 @@
 namespace fp4 {
 
 __device__ int g_status = 0;
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(static_cast<unsigned long long>(n)); }
 
 int num_sms() {
   static int cached[64] = {0};
@@ -69,6 +73,7 @@ static int check_out(const fp4_qtensor* out) {
   if (!out || !out->codes || !out->tensor_scale || (!out->scales && !out->scales_swz))
     return FP4_ERR_INVALID_ARG;
   if (!aligned(out->codes, 16) || (out->scales_swz && !aligned(out->scales_swz, 16)) ||
+      (out->scales && !aligned(out->scales, 16)) || (out->mask && !aligned(out->mask, 16)) ||
       !aligned(out->tensor_scale, 4))
     return FP4_ERR_ALIGNMENT;
   return FP4_OK;
@@ -87,6 +92,7 @@ static int launch_pad(uint8_t* swz, int64_t rows, int64_t ng, cudaStream_t s) {
   int64_t blocks = (n + 255) / 256;
   if (blocks > 4096) blocks = 4096;
   k_swz_pad<<<unsigned(blocks), 256, 0, s>>>(swz, rows, ng, nkb);
+  count_launch();
   return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
@@ -126,6 +132,7 @@ static int run_quant(int load, int fmt, int rnd, int had, QParams& p, void* ws, 
       case 32: k_eden_pass2<32><<<unsigned(blocks), 256, 0, s>>>(p); break;
       default: k_eden_pass2<128><<<unsigned(blocks), 256, 0, s>>>(p); break;
     }
+    count_launch();
     if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
   }
   return launch_pad(p.swz, p.rows, p.cols / (fmt == FP4_NVFP4 ? 16 : 32), s);
@@ -226,6 +233,7 @@ int fp4_hadamard(const void* x, float* y, int64_t rows, int64_t cols, fp4_had ha
     case 32: k_hadamard<32><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
     default: k_hadamard<128><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
   }
+  count_launch();
   return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
@@ -238,6 +246,7 @@ int fp4_swizzle_scales(const uint8_t* scales, int64_t rows, int64_t n_groups, ui
   int64_t nkb = (n_groups + 3) / 4, n = rows * n_groups, blocks = (n + 255) / 256;
   if (blocks > 4096) blocks = 4096;
   k_swizzle<<<unsigned(blocks), 256, 0, s>>>(scales, rows, n_groups, nkb, swz);
+  count_launch();
   if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
   return launch_pad(swz, rows, n_groups, s);
 }
@@ -254,6 +263,16 @@ int fp4_get_last_error(fp4_stream_t stream) {
     cudaMemcpy(a, &z, sizeof(int), cudaMemcpyHostToDevice);
   }
   return v;
+}
+
+unsigned long long fp4_launch_count(void) { return g_launches.load(); }
+
+int fp4_selftest_e2m1(unsigned long long* mismatches, fp4_stream_t stream) {
+  if (!mismatches) return FP4_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  k_selftest_e2m1<<<unsigned(num_sms() * 8), 256, 0, s>>>(mismatches);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
 const char* fp4_status_string(int st) {

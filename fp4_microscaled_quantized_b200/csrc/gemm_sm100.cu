@@ -7,11 +7,15 @@
 // the Quartet backward correction dx = 16/9 H32^-1(dx_q (.) (1 - M)) (the 16/9
 // is the product of the two 4/3 tensor scales).
 //
-// Structure: persistent CTAs (one per SM), 128 x 256 output tiles, a 4-stage
+// Structure: persistent CTAs (one per SM), 128 x 256 output tiles, a 3-stage
 // shared-memory ring fed by TMA (codes, 128-byte swizzle) and bulk copies
 // (scale atoms, already in the tensor-core layout), warp roles:
 //   warp 0  TMA producer          warp 1  MMA issuer (one thread)
-//   warp 2  TMEM allocator        warps 4-7  epilogue (TMEM -> registers -> HBM)
+//   warp 2  TMEM allocator        warps 4-7  epilogue (TMEM -> smem -> TMA store)
+//   warps 8-11  scale-factor stagers: each writes its TMEM lane quadrant of the
+//   scales with tcgen05.st into one of two TMEM buffers, so the MMA issue queue
+//   holds only MMAs (copying scales with tcgen05.cp from the MMA thread
+//   serialises them with the MMAs and halves throughput).
 // Every mbarrier wait is bounded; on timeout the kernel records
 // FP4_ERR_TIMEOUT, stops issuing work, frees its TMEM and returns.
 #include <cuda.h>
@@ -28,16 +32,19 @@ int num_sms();
 namespace gemm {
 
 constexpr int BM = 128, BN = 256, BK = 256;         // BK in FP4 elements (128 bytes)
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BK / 2;                 // 16 KB
 constexpr int B_BYTES = BN * BK / 2;                 // 32 KB
 constexpr int SFA_BYTES = 4 * 512;                   // up to 4 atoms (NVFP4)
 constexpr int SFB_BYTES = 8 * 512;                   // 2 row blocks x 4 atoms
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr int THREADS = 256;
+constexpr int STG_BYTES = BM * 128;                  // epilogue staging: 128 rows x 128 bytes
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * STG_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int THREADS = 384;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_COL = 0, SFA_COL = 256, SFB_COL = 272;
+// TMEM columns: the accumulator, then two scale-factor buffers (SFA 16 + SFB
+// 32 columns each) so the stagers fill one while the MMAs read the other.
+constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_BUF_COLS = 48, SFB_OFF = 16;
 constexpr unsigned long long WAIT_LIMIT = 4000000000ull;  // ~2 s of SM clocks
 
 enum : int { OUT_F32 = 0, OUT_BF16 = 1 };
@@ -117,6 +124,31 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
+// TMA store of a staged tile (bulk-group completion) and its bookkeeping.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// OR of a predicate over the 128 epilogue threads (named barrier 1).
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v))
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -135,20 +167,6 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
   d |= uint64_t(1) << 46;
   d |= uint64_t(2) << 61;
   return d;
-}
-
-// Scale atom source for tcgen05.cp: 32 rows x 16 bytes, no swizzle, 8-row
-// core matrices 128 B apart.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= uint64_t((saddr >> 4) & 0x3FFF);
-  d |= uint64_t(128 >> 4) << 32;
-  d |= uint64_t(1) << 46;
-  return d;
-}
-
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
 template <int FMT>
@@ -211,18 +229,22 @@ __device__ __forceinline__ void tile_coords(int64_t t, int64_t nm, int64_t nn, i
 // ---------------------------------------------------------------- kernel --
 template <int FMT, int OUT, int EPI>
 __global__ void __launch_bounds__(THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, Params p) {
+    k_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+           const __grid_constant__ CUtensorMap map_d, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_BYTES;
   uint8_t* sSFA = sB + STAGES * B_BYTES;
   uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+  uint8_t* sStage = sSFB + STAGES * SFB_BYTES;         // 1024-byte aligned (stage sizes are)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStage + 2 * STG_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* sf_full = acc_empty + 1;
+  uint64_t* sf_empty = sf_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -234,6 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 128);
+    for (int b = 0; b < 2; ++b) { mbar_init(&sf_full[b], 128); mbar_init(&sf_empty[b], 1); }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -275,103 +298,174 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // --------------------------------------------------------- MMA issue --
-    int s = 0;
+    // Walks this CTA's (tile, k-tile) sequence; k-tile i uses operand stage
+    // i % STAGES and scale buffer i % 2.
+    int s = 0, buf = 0;
     uint32_t ph = 0, acc_ph = 0;
-    for (int64_t t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+    int use[2] = {0, 0};
+    bool ok = true;
+    for (int64_t t = blockIdx.x; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
       if (!mbar_wait(acc_empty, acc_ph ^ 1, abort_flag, p.status)) break;
       tc_fence_after();
-      bool ok = true;
       for (int64_t kt = 0; kt < nkt; ++kt) {
         if (!mbar_wait(&full[s], ph, abort_flag, p.status)) { ok = false; break; }
+        if (!mbar_wait(&sf_full[buf], uint32_t(use[buf] & 1), abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
         const int n_mma = kel / 64;
-        const int atoms = FMT == 1 ? n_mma : (n_mma + 1) / 2;
         const uint32_t a_base = smem_u32(sA + s * A_BYTES), b_base = smem_u32(sB + s * B_BYTES);
-        for (int a = 0; a < atoms; ++a) {
-          tc_cp_sf(tmem + SFA_COL + 4 * a, desc_sf(smem_u32(sSFA + s * SFA_BYTES + a * 512)));
-          tc_cp_sf(tmem + SFB_COL + 8 * a, desc_sf(smem_u32(sSFB + s * SFB_BYTES + a * 512)));
-          tc_cp_sf(tmem + SFB_COL + 8 * a + 4, desc_sf(smem_u32(sSFB + s * SFB_BYTES + (4 + a) * 512)));
-        }
+        const uint32_t sfbase = tmem + SF_COL + SF_BUF_COLS * uint32_t(buf);
         for (int kk = 0; kk < n_mma; ++kk) {
           const int atom = FMT == 1 ? kk : kk / 2;
           const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
-          const uint32_t sfa = (tmem + SFA_COL + 4 * atom) | (sf_id << 30);
-          const uint32_t sfb = (tmem + SFB_COL + 8 * atom) | (sf_id << 30);
+          const uint32_t sfa = (sfbase + 4 * atom) | (sf_id << 30);
+          const uint32_t sfb = (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30);
           tc_mma<FMT>(tmem + ACC_COL, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
                       idesc(FMT, BN, BM, sf_id, sf_id), sfa, sfb, (kt > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&empty[s]);
+        tc_commit(&sf_empty[buf]);
+        if (kt == nkt - 1) tc_commit(acc_full);
+        ++use[buf];
+        buf ^= 1;
         if (++s == STAGES) { s = 0; ph ^= 1; }
       }
-      if (!ok) break;
-      tc_commit(acc_full);
       acc_ph ^= 1;
     }
-  } else if (warp >= 4) {
-    // ---------------------------------------------------------- epilogue --
+  } else if (warp >= 8) {
+    // ------------------------------------------- scale factors -> TMEM --
+    // Lane l of warp q copies row l of every scale atom of the stage (16 bytes
+    // = the scales of rows l, l+32, l+64, l+96) into TMEM lane 32q + l: the
+    // same replicated layout tcgen05.cp .32x128b.warpx4 produces.
     const int q = warp & 3;
+    int s = 0, buf = 0;
+    uint32_t ph = 0;
+    int use[2] = {0, 0};
+    bool ok = true;
+    for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+      for (int64_t kt = 0; kt < nkt; ++kt) {
+        const bool a = mbar_wait(&sf_empty[buf], uint32_t(use[buf] & 1) ^ 1u, abort_flag, p.status);
+        const bool b = a && mbar_wait(&full[s], ph, abort_flag, p.status);
+        if (__any_sync(0xFFFFFFFFu, !b)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t va[16], vb[32];
+        const uint8_t* sa = sSFA + s * SFA_BYTES + lane * 16;
+        const uint8_t* sb = sSFB + s * SFB_BYTES + lane * 16;
+#pragma unroll
+        for (int at = 0; at < 4; ++at) {
+          const uint4 x = *reinterpret_cast<const uint4*>(sa + at * 512);
+          va[4 * at] = x.x; va[4 * at + 1] = x.y; va[4 * at + 2] = x.z; va[4 * at + 3] = x.w;
+#pragma unroll
+          for (int rb = 0; rb < 2; ++rb) {
+            const uint4 y = *reinterpret_cast<const uint4*>(sb + (rb * 4 + at) * 512);
+            const int o = 8 * at + 4 * rb;
+            vb[o] = y.x; vb[o + 1] = y.y; vb[o + 2] = y.z; vb[o + 3] = y.w;
+          }
+        }
+        const uint32_t base = tmem + (uint32_t(q * 32) << 16) + SF_COL + SF_BUF_COLS * uint32_t(buf);
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(base),
+            "r"(va[0]), "r"(va[1]), "r"(va[2]), "r"(va[3]), "r"(va[4]), "r"(va[5]), "r"(va[6]), "r"(va[7]), "r"(va[8]),
+            "r"(va[9]), "r"(va[10]), "r"(va[11]), "r"(va[12]), "r"(va[13]), "r"(va[14]), "r"(va[15]));
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+            "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(base + SFB_OFF),
+            "r"(vb[0]), "r"(vb[1]), "r"(vb[2]), "r"(vb[3]), "r"(vb[4]), "r"(vb[5]), "r"(vb[6]), "r"(vb[7]), "r"(vb[8]),
+            "r"(vb[9]), "r"(vb[10]), "r"(vb[11]), "r"(vb[12]), "r"(vb[13]), "r"(vb[14]), "r"(vb[15]), "r"(vb[16]),
+            "r"(vb[17]), "r"(vb[18]), "r"(vb[19]), "r"(vb[20]), "r"(vb[21]), "r"(vb[22]), "r"(vb[23]), "r"(vb[24]),
+            "r"(vb[25]), "r"(vb[26]), "r"(vb[27]), "r"(vb[28]), "r"(vb[29]), "r"(vb[30]), "r"(vb[31]));
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(&sf_full[buf]);
+        ++use[buf];
+        buf ^= 1;
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------- epilogue --
+    // TMEM -> registers -> (scale, Quartet mask + H32^-1) -> 128-byte-swizzled
+    // staging in shared memory -> TMA store.  The accumulator is released as
+    // soon as its last columns are in registers, so the next tile's MMAs
+    // overlap the stores.
+    constexpr int CW = OUT == OUT_F32 ? 32 : 64;       // columns per 128-byte staged row
+    const int q = warp & 3, tid = threadIdx.x - 128, rl = q * 32 + lane;
     uint32_t acc_ph = 0;
+    int chunk = 0;
     const float tscale = __fmul_rn(*p.ta, *p.tb);
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
       int64_t mb, nb;
       tile_coords(t, nm, nn, mb, nb);
-      if (!mbar_wait(acc_full, acc_ph, abort_flag, p.status)) break;
+      const bool got = mbar_wait(acc_full, acc_ph, abort_flag, p.status);
+      if (epi_any(!got)) break;                         // uniform decision across the 4 warps
       acc_ph ^= 1;
       tc_fence_after();
-      const int64_t row = mb * BM + q * 32 + lane;
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem + ACC_COL + (uint32_t(q * 32) << 16) + c * 32, v);
-        const int64_t col0 = nb * BN + c * 32;
-        if (row >= p.M || col0 >= p.N) continue;
+      const int64_t row = mb * BM + rl;
+      for (int c = 0; c < BN / CW; ++c) {
+        float v[CW];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = v[j] * tscale;
+        for (int i = 0; i < CW / 32; ++i)
+          tmem_ld32(tmem + ACC_COL + (uint32_t(q * 32) << 16) + c * CW + 32 * i, v + 32 * i);
+        if (c == BN / CW - 1) {                         // accumulator fully read: release it
+          tc_fence_before();
+          mbar_arrive(acc_empty);
+        }
+        const int64_t col0 = nb * BN + c * CW;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) v[j] = v[j] * tscale;
         if (EPI == 1) {
-          if (p.mask) {
-            uint32_t mw = *reinterpret_cast<const uint32_t*>(p.mask + row * (p.N >> 3) + (col0 >> 3));
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if ((mw >> j) & 1u) v[j] = 0.0f;
-          }
+          for (int hb = 0; hb < CW / 32; ++hb) {
+            float* u = v + 32 * hb;
+            const int64_t cb = col0 + 32 * hb;
+            if (p.mask && row < p.M && cb < p.N) {
+              const uint32_t mw = *reinterpret_cast<const uint32_t*>(p.mask + row * (p.N >> 3) + (cb >> 3));
 #pragma unroll
-          for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (i & h) continue;
-              float a = v[i], b = v[i + h];
-              v[i] = a + b;
-              v[i + h] = a - b;
+              for (int j = 0; j < 32; ++j)
+                if ((mw >> j) & 1u) u[j] = 0.0f;
             }
-          }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= 0.176776695296636881f;
+            for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                if (i & h) continue;
+                float a = u[i], b = u[i + h];
+                u[i] = a + b;
+                u[i + h] = a - b;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] *= 0.176776695296636881f;
+          }
         }
-        const int ncols = int(p.N - col0 < 32 ? p.N - col0 : 32);
+        uint32_t wds[32];
         if (OUT == OUT_F32) {
-          float* dst = static_cast<float*>(p.D) + row * p.N + col0;
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            if (j < ncols) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          for (int j = 0; j < 32; ++j) wds[j] = __float_as_uint(v[j]);
         } else {
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.D) + row * p.N + col0;
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            if (j >= ncols) continue;
-            uint4 w;
-            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(v[j + 2 * i], v[j + 2 * i + 1]);
-              wp[i] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            *reinterpret_cast<uint4*>(dst + j) = w;
+          for (int j = 0; j < 32; ++j) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            wds[j] = *reinterpret_cast<uint32_t*>(&h2);
           }
         }
+        uint8_t* stg = sStage + (chunk & 1) * STG_BYTES;
+        if (tid == 0) bulk_wait_read1();                // the store that last used this buffer has read it
+        epi_bar();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)                     // 16-byte chunk j of row rl, 128B-swizzled
+          *reinterpret_cast<uint4*>(stg + rl * 128 + ((j ^ (rl & 7)) << 4)) =
+              make_uint4(wds[4 * j], wds[4 * j + 1], wds[4 * j + 2], wds[4 * j + 3]);
+        fence_proxy_async();
+        epi_bar();
+        if (tid == 0) {
+          tma_store_2d(&map_d, stg, int(col0), int(mb * BM));
+          bulk_commit();
+        }
+        ++chunk;
       }
-      tc_fence_before();
-      mbar_arrive(acc_empty);
     }
+    if (tid == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -414,8 +508,25 @@ static bool make_map(CUtensorMap* m, const void* codes, int64_t rows, int64_t K,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output D (M x N, fp32 or bf16) for the epilogue's TMA stores: box of 128
+// bytes x 128 rows, 128-byte swizzle (the staging layout); out-of-range rows
+// and columns of a tile are not written.
+static bool make_map_d(CUtensorMap* m, void* D, int64_t M, int64_t N, int out_dtype) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int es = out_dtype ? 2 : 4;
+  cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(M)};
+  cuuint64_t strides[1] = {cuuint64_t(N) * cuuint64_t(es)};
+  cuuint32_t box[2] = {cuuint32_t(128 / es), cuuint32_t(BM)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, out_dtype ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, D, dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int FMT, int OUT, int EPI>
-static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
+                          cudaStream_t s) {
   auto kern = k_gemm<FMT, OUT, EPI>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -427,7 +538,8 @@ static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const Pa
   }
   int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
   int grid = int(tiles < num_sms() ? tiles : num_sms());
-  kern<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+  kern<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mb, md, p);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -460,8 +572,9 @@ extern "C" int fp4_gemm(const fp4_qtensor* A, const fp4_qtensor* B, void* D, int
     size_t bytes = size_t(M) * size_t(N) * (out_dtype ? 2 : 4);
     return cudaMemsetAsync(D, 0, bytes, s) == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
   }
-  CUtensorMap ma, mb;
-  if (!gemm::make_map(&ma, A->codes, M, K, gemm::BM) || !gemm::make_map(&mb, B->codes, N, K, gemm::BN))
+  CUtensorMap ma, mb, md;
+  if (!gemm::make_map(&ma, A->codes, M, K, gemm::BM) || !gemm::make_map(&mb, B->codes, N, K, gemm::BN) ||
+      !gemm::make_map_d(&md, D, M, N, out_dtype))
     return FP4_ERR_CUDA;
   gemm::Params p{};
   p.M = M; p.N = N; p.K = K;
@@ -472,11 +585,11 @@ extern "C" int fp4_gemm(const fp4_qtensor* A, const fp4_qtensor* B, void* D, int
   cudaError_t e;
   const bool nv = A->fmt == FP4_NVFP4, bf = out_dtype == 1, epi = epi_inverse_had == 32;
   if (nv) {
-    if (bf) e = epi ? gemm::launch<1, 1, 1>(ma, mb, p, s) : gemm::launch<1, 1, 0>(ma, mb, p, s);
-    else e = epi ? gemm::launch<1, 0, 1>(ma, mb, p, s) : gemm::launch<1, 0, 0>(ma, mb, p, s);
+    if (bf) e = epi ? gemm::launch<1, 1, 1>(ma, mb, md, p, s) : gemm::launch<1, 1, 0>(ma, mb, md, p, s);
+    else e = epi ? gemm::launch<1, 0, 1>(ma, mb, md, p, s) : gemm::launch<1, 0, 0>(ma, mb, md, p, s);
   } else {
-    if (bf) e = epi ? gemm::launch<0, 1, 1>(ma, mb, p, s) : gemm::launch<0, 1, 0>(ma, mb, p, s);
-    else e = epi ? gemm::launch<0, 0, 1>(ma, mb, p, s) : gemm::launch<0, 0, 0>(ma, mb, p, s);
+    if (bf) e = epi ? gemm::launch<0, 1, 1>(ma, mb, md, p, s) : gemm::launch<0, 1, 0>(ma, mb, md, p, s);
+    else e = epi ? gemm::launch<0, 0, 1>(ma, mb, md, p, s) : gemm::launch<0, 0, 0>(ma, mb, md, p, s);
   }
   return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

@@ -1,0 +1,481 @@
+// Fast path of the quantiser: 32 consecutive elements of one output row per
+// lane (used when the inner dimension is a multiple of 32).  Scale groups (16
+// or 32) and rotation blocks up to 32 live entirely in one lane's registers;
+// a 128-block spans 4 aligned lanes, so the FWHT needs two shuffle stages and
+// the MS-EDEN sums two.  Arithmetic is element-for-element the same as the
+// 8-per-lane path in quant_kernels.cuh (same butterfly order, same pairwise
+// trees), so both produce identical bits.
+#pragma once
+#include "quant_kernels.cuh"
+
+namespace fp4 {
+
+// E2M1 RTN of 8 values into one word (element j in bits 4j..4j+3) with the
+// hardware conversion (round to nearest even, saturating at +-6); negative
+// zeros are then cleared so a value rounding to 0 encodes as +0.
+__device__ __forceinline__ uint32_t enc8_hw(const float* v) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(w)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  const uint32_t nz = ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;  // bit 3 set iff mag != 0
+  return w & (nz | 0x77777777u);
+}
+
+// Software reference of the same word (the per-element encoder).
+__device__ __forceinline__ uint32_t enc8_sw(const float* v) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) w |= e2m1_rtn(v[j]) << (4 * j);
+  return w;
+}
+
+// Grid value of an E2M1 code from its bits: magnitude m >= 2 is 2^((m>>1)-1)
+// (1 + (m&1)/2), i.e. fp32 bits (m << 22) + 0x3F000000; m = 1 is 0.5.
+__device__ __forceinline__ float e2m1_dec(uint32_t c) {
+  const uint32_t m = c & 7u;
+  uint32_t b = (m << 22) + 0x3F000000u - (m == 1u ? 0x400000u : 0u);
+  b = m ? b : 0u;
+  return bitsf(b | ((c & 8u) << 28));
+}
+
+__device__ __forceinline__ float tree16(const float* s) { return __fadd_rn(tree8(s), tree8(s + 8)); }
+__device__ __forceinline__ float tree32(const float* s) { return __fadd_rn(tree16(s), tree16(s + 16)); }
+
+// 16 codes of x * inv (or zeros when !ok) into two words.
+__device__ __forceinline__ void enc16(const float* x, float inv, bool ok, uint32_t* w) {
+  float v[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(x[j], inv);
+  w[0] = ok ? enc8_hw(v) : 0u;
+  w[1] = ok ? enc8_hw(v + 8) : 0u;
+}
+
+// fp32 squared error of 16 elements against codes * d, pairwise tree.
+__device__ __forceinline__ float sse16(const float* x, const uint32_t* w, float d) {
+  float s[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    float e = __fsub_rn(x[j], __fmul_rn(e2m1_dec(w[j >> 3] >> (4 * (j & 7))), d));
+    s[j] = __fmul_rn(e, e);
+  }
+  return tree16(s);
+}
+
+// Block FWHT over HAD consecutive elements, 32 per lane (HAD / 32 aligned
+// lanes for HAD = 128), same butterfly order as fwht8_lanes.
+template <int HAD>
+__device__ __forceinline__ void fwht32_lanes(float* x, uint32_t sign, int lane) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if ((sign >> j) & 1u) x[j] = -x[j];
+  constexpr int HIN = HAD < 32 ? HAD : 32;
+#pragma unroll
+  for (int h = 1; h < HIN; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i & h) continue;
+      float a = x[i], b = x[i + h];
+      x[i] = __fadd_rn(a, b);
+      x[i + h] = __fsub_rn(a, b);
+    }
+  }
+#pragma unroll
+  for (int hl = 1; hl < HAD / 32; hl <<= 1) {
+    const bool upper = (lane & hl) != 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float o = __shfl_xor_sync(0xFFFFFFFFu, x[i], hl);
+      x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+    }
+  }
+  const float c = HAD == 16 ? 0.25f : (HAD == 32 ? 0.176776695296636881f : 0.0883883476483184405f);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], c);
+}
+
+template <int FMT, int RND, int HAD>
+__device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t orow, int64_t ocol, int lane,
+                                              const QParams& p, const Shared& sh, uint32_t amax_in) {
+  constexpr int G = FMT == FMT_NV ? 16 : 32;
+  constexpr int NG = 32 / G;
+  if (HAD > 0) {
+    uint32_t sign = 0;
+    if (p.randomized) {
+      if (HAD == 16) {
+        sign = sh.signs[0] & 0xFFFFu;
+        sign |= sign << 16;
+      } else {
+        sign = sh.signs[int(ocol & (HAD - 1)) >> 5];
+      }
+    }
+    fwht32_lanes<HAD>(x, sign, lane);
+  }
+  uint32_t gmb[NG];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < G; ++j) m = max(m, absbits(x[g * G + j]));
+    gmb[g] = m;
+  }
+  uint32_t lmax = NG == 2 ? max(gmb[0], gmb[NG - 1]) : gmb[0];
+  if (!active) lmax = 0;
+  if (RND == R_AMAX) return lmax;
+  if (active && lmax >= 0x7F800000u && (FMT == FMT_MX || RND == R_EDEN)) flag_status(p.status, ST_NONFINITE);
+
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  uint32_t sb[NG];
+  uint32_t mbits = 0;
+
+  if (FMT == FMT_NV && (RND == R_RTN || RND == R_FOS || RND == R_SR || RND == R_QUEST)) {
+    const float s32 = nv_tensor_scale(amax_in, RND == R_SR ? FP4_NV_SR_DIV : FP4_NV_RTN_DIV);
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      const float* xg = x + 16 * g;
+      const float gmax = bitsf(gmb[g]);
+      uint32_t* wg = w + 2 * g;
+      if (RND == R_RTN) {
+        uint32_t s8 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 6.0f)));
+        float d = __fmul_rn(e4m3_value(s8), s32), inv = __frcp_rn(d);
+        enc16(xg, inv, finite_pos(d, inv), wg);
+        sb[g] = s8;
+      } else if (RND == R_FOS) {
+        uint32_t s6 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 6.0f)));
+        uint32_t s4 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 4.0f)));
+        float d6 = __fmul_rn(e4m3_value(s6), s32), i6 = __frcp_rn(d6);
+        float d4 = __fmul_rn(e4m3_value(s4), s32), i4 = __frcp_rn(d4);
+        uint32_t w6[2], w4[2];
+        enc16(xg, i6, finite_pos(d6, i6), w6);
+        enc16(xg, i4, finite_pos(d4, i4), w4);
+        const bool pick4 = sse16(xg, w4, d4) < sse16(xg, w6, d6);
+        wg[0] = pick4 ? w4[0] : w6[0];
+        wg[1] = pick4 ? w4[1] : w6[1];
+        sb[g] = pick4 ? s4 : s6;
+      } else if (RND == R_SR) {
+        uint32_t s8 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, FP4_NV_SR_GDIV)));
+        float d = __fmul_rn(e4m3_value(s8), s32), inv = __frcp_rn(d);
+        const bool ok = finite_pos(d, inv);
+        const uint64_t q0 = uint64_t(orow * p.cols + ocol + 16 * g) >> 2;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          u32x4 r = philox_block(p.seed, q0 + b, TAG_SR_ELEM, p.tensor_tag);
+          const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = 4 * b + j;
+            uint32_t c = ok ? e2m1_sr(__fmul_rn(xg[e], inv), u24(rw[j])) : 0u;
+            wg[e >> 3] |= c << (4 * (e & 7));
+          }
+        }
+        sb[g] = s8;
+      } else {  // QuEST on the E4M3 scale grid
+        float sq[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) sq[j] = __fmul_rn(xg[j], xg[j]);
+        const float sig2 = __fdiv_rn(tree16(sq), 16.0f);
+        const float hi = __fmul_rn(25.0f, sig2);
+        auto t2 = [&](int cc) {
+          float t = __fmul_rn(6.0f, __fmul_rn(e4m3_value(uint32_t(cc)), s32));
+          return __fmul_rn(t, t);
+        };
+        int lo = 1, hi_i = 127;
+        while (lo < hi_i) { int mid = (lo + hi_i) >> 1; if (t2(mid) >= sig2) hi_i = mid; else lo = mid + 1; }
+        const int clo = lo;
+        lo = 0; hi_i = 126;
+        while (lo < hi_i) { int mid = (lo + hi_i + 1) >> 1; if (t2(mid) <= hi) lo = mid; else hi_i = mid - 1; }
+        const int chi = lo;
+        uint32_t s8;
+        if (clo <= chi && chi >= 1) {
+          float best = __int_as_float(0x7F800000);
+          int bc = clo;
+          for (int cc = clo; cc <= chi; ++cc) {
+            float d = __fmul_rn(e4m3_value(uint32_t(cc)), s32), inv = __frcp_rn(d);
+            uint32_t wt[2];
+            enc16(xg, inv, finite_pos(d, inv), wt);
+            float e = sse16(xg, wt, d);
+            if (e <= best) { best = e; bc = cc; }
+          }
+          s8 = uint32_t(bc);
+        } else {
+          s8 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 6.0f)));
+        }
+        float d = __fmul_rn(e4m3_value(s8), s32), inv = __frcp_rn(d);
+        const bool ok = finite_pos(d, inv);
+        enc16(xg, inv, ok, wg);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          mbits |= uint32_t(ok && fabsf(__fmul_rn(xg[j], inv)) > 6.0f) << (16 * g + j);
+        sb[g] = s8;
+      }
+    }
+  } else if (FMT == FMT_NV && RND == R_EDEN) {
+    float num_g[NG], den_g[NG];
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      const float* xg = x + 16 * g;
+      const float pq = e8m3_round(__fdiv_rn(bitsf(gmb[g]), FP4_EDEN_S));
+      const float inv = __frcp_rn(pq);
+      enc16(xg, inv, finite_pos(pq, inv), w + 2 * g);
+      float yy[16], yq[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        yy[j] = __fmul_rn(xg[j], xg[j]);
+        yq[j] = __fmul_rn(xg[j], __fmul_rn(e2m1_dec(w[2 * g + (j >> 3)] >> (4 * (j & 7))), pq));
+      }
+      num_g[g] = tree16(yy);       // the two halves of the 32-element tree
+      den_g[g] = tree16(yq);
+      sb[g] = fbits(pq) >> 16;     // bf16 pseudo-scale (exact)
+    }
+    if (active) {
+      *reinterpret_cast<uint32_t*>(p.pseudo + orow * (p.cols >> 4) + (ocol >> 4)) = sb[0] | (sb[NG - 1] << 16);
+    }
+    if (HAD == 16) {
+      float S2[2];
+#pragma unroll
+      for (int g = 0; g < 2; ++g) S2[g] = den_g[g] > 0.0f ? __fdiv_rn(num_g[g], den_g[g]) : 1.0f;
+      if (active) *reinterpret_cast<float2*>(p.eden_S + orow * (p.cols >> 4) + (ocol >> 4)) = make_float2(S2[0], S2[1]);
+    } else {
+      float num = __fadd_rn(num_g[0], num_g[NG - 1]), den = __fadd_rn(den_g[0], den_g[NG - 1]);
+      if (HAD == 128) {
+        num = tree_lanes<4>(num);
+        den = tree_lanes<4>(den);
+      }
+      const float S = den > 0.0f ? __fdiv_rn(num, den) : 1.0f;
+      if (active && (HAD == 32 || (lane & 3) == 0)) p.eden_S[orow * (p.cols / HAD) + ocol / HAD] = S;
+    }
+  } else if (FMT == FMT_MX && (RND == R_RTN || RND == R_SR)) {
+    int e = int(gmb[0] >> 23) - 129;
+    e = e < -127 ? -127 : e;
+    const float sc = pow2f(-e);
+    if (RND == R_RTN) {
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(x[j], sc);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) w[k] = enc8_hw(v + 8 * k);
+    } else {
+      const uint64_t q0 = uint64_t(orow * p.cols + ocol) >> 2;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        u32x4 r = philox_block(p.seed, q0 + b, TAG_SR_ELEM, p.tensor_tag);
+        const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int el = 4 * b + j;
+          uint32_t c = e2m1_sr(__fmul_rn(__fmul_rn(x[el], FP4_QUARTET_PRESCALE), sc), u24(rw[j]));
+          w[el >> 3] |= c << (4 * (el & 7));
+        }
+      }
+    }
+    sb[0] = uint32_t(e + 127);
+  } else if (FMT == FMT_MX && RND == R_QUEST) {
+    float sq[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) sq[j] = __fmul_rn(x[j], x[j]);
+    const float sig2 = __fdiv_rn(tree32(sq), 32.0f);
+    const float hi = __fmul_rn(25.0f, sig2);
+    const int fl = sig2 > 0.0f ? floor_log2(sig2) : -300;
+    const int elo = (fl >> 1) - 4;
+    int be = 0;
+    float bs = __int_as_float(0x7F800000);
+    bool found = false;
+#pragma unroll 1
+    for (int k = 0; k < 8; ++k) {
+      int e = elo + k;
+      e = e < -127 ? -127 : (e > 125 ? 125 : e);
+      const float t = __fmul_rn(6.0f, pow2f(e));
+      const float tt = __fmul_rn(t, t);
+      const bool inwin = (sig2 <= tt) && (tt <= hi) && (sig2 > 0.0f);
+      if (!inwin) continue;              // (an out-of-window candidate never wins)
+      const float sc = pow2f(-e), d = pow2f(e);
+      uint32_t wt[4];
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(x[j], sc);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) wt[q] = enc8_hw(v + 8 * q);
+      const float s = __fadd_rn(sse16(x, wt, d), sse16(x + 16, wt + 2, d));
+      if (s <= bs) { bs = s; be = e; }
+      found = true;
+    }
+    int e;
+    if (found) {
+      e = be;
+    } else {
+      e = int(gmb[0] >> 23) - 129;
+      e = e < -127 ? -127 : e;
+    }
+    const float sc = pow2f(-e);
+    float v[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      v[j] = __fmul_rn(x[j], sc);
+      mbits |= uint32_t(fabsf(v[j]) > 6.0f) << j;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = enc8_hw(v + 8 * q);
+    sb[0] = uint32_t(e + 127);
+  }
+
+  if (active) {
+    *reinterpret_cast<uint4*>(p.codes + orow * (p.cols >> 1) + (ocol >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (RND != R_EDEN) {
+      const int64_t k = ocol / G;
+      if (NG == 2) {
+        const uint16_t two = uint16_t(sb[0] | (sb[NG - 1] << 8));
+        if (p.scales) *reinterpret_cast<uint16_t*>(p.scales + orow * (p.cols / G) + k) = two;
+        if (p.swz) *reinterpret_cast<uint16_t*>(p.swz + swz_offset(orow, k, p.nkb)) = two;
+      } else {
+        if (p.scales) p.scales[orow * (p.cols / G) + k] = uint8_t(sb[0]);
+        if (p.swz) p.swz[swz_offset(orow, k, p.nkb)] = uint8_t(sb[0]);
+      }
+    }
+    if (RND == R_QUEST && p.mask) *reinterpret_cast<uint32_t*>(p.mask + orow * (p.cols >> 3) + (ocol >> 3)) = mbits;
+  }
+  return lmax;
+}
+
+// Row-wise, 32 elements per lane, grid-stride over 32-element tasks.
+template <int LOAD, int FMT, int RND, int HAD>
+__global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
+  __shared__ Shared sh;
+  load_signs<HAD>(sh, p);
+  const int lane = threadIdx.x & 31;
+  const int64_t tpr = p.cols >> 5, tasks = p.rows * tpr;
+  const uint32_t amax_in = (FMT == FMT_NV && RND != R_EDEN && RND != R_AMAX) ? *p.amax_bits : 0u;
+  const float in_ts = LOAD == LD_ROW_FP4 ? *p.in_ts : 1.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) write_tensor_scale<FMT, RND>(p, amax_in);
+  uint32_t acc = 0;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t base = int64_t(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); base < tasks; base += stride) {
+    const int64_t t = base + lane;
+    const bool active = t < tasks;
+    const int64_t orow = active ? t / tpr : 0, ocol = active ? (t % tpr) * 32 : 0;
+    float x[32];
+    if (LOAD == LD_ROW) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + orow * p.cols + ocol);
+      uint4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = active ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bf16x8_to_f32(v[i], x + 8 * i);
+    } else {
+      uint4 cw = make_uint4(0, 0, 0, 0);
+      uint32_t s0 = 0, s1 = 0;
+      const int gin = p.in_fmt == FMT_NV ? 16 : 32;
+      if (active) {
+        cw = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) + orow * (p.cols >> 1) + (ocol >> 1)));
+        s0 = p.in_scales[orow * (p.cols / gin) + ocol / gin];
+        s1 = p.in_scales[orow * (p.cols / gin) + (ocol + 16) / gin];
+      }
+      const float sa = fp4_in_scale(s0, p.in_fmt), sbv = fp4_in_scale(s1, p.in_fmt);
+      const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        x[j] = __fmul_rn(__fmul_rn(e2m1_dec(cws[j >> 3] >> (4 * (j & 7))), j < 16 ? sa : sbv), in_ts);
+    }
+    acc = max(acc, process32<FMT, RND, HAD>(x, active, orow, ocol, lane, p, sh, amax_in));
+  }
+  if (RND == R_AMAX || RND == R_EDEN) block_max_atomic(acc, sh, p.amax_bits, p.status);
+}
+
+// Transposed, 32 elements per lane: the 128 x 64 input tile is staged as fp32
+// with a 4-float skew every 32 columns, so the 16-byte reads of four lanes on
+// one 128-element output row hit distinct banks.
+constexpr int T32_PITCH = 144;
+__device__ __forceinline__ int t32_col(int c) { return c + 4 * (c >> 5); }
+
+template <int LOAD, int FMT, int RND, int HAD>
+__global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
+  __shared__ Shared sh;
+  __shared__ __align__(16) float tile[TR_IN_COLS][T32_PITCH];
+  load_signs<HAD>(sh, p);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t r0 = int64_t(blockIdx.x) * TR_IN_ROWS, c0 = int64_t(blockIdx.y) * TR_IN_COLS;
+  const int64_t R = p.in_rows, C = p.in_cols;
+  {
+    const int rh = w >> 2, cb = w & 3;
+    const int rl = 64 * rh + 2 * lane;
+    const int64_t cc = c0 + 16 * cb;
+    float va[16], vb[16];
+    if (LOAD == LD_TRANS) {
+      const uint16_t* xb = static_cast<const uint16_t*>(p.x);
+      uint4 a[2], b[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t col = cc + 8 * h;
+        a[h] = (col < C && r0 + rl < R) ? __ldg(reinterpret_cast<const uint4*>(xb + (r0 + rl) * C + col))
+                                        : make_uint4(0, 0, 0, 0);
+        b[h] = (col < C && r0 + rl + 1 < R) ? __ldg(reinterpret_cast<const uint4*>(xb + (r0 + rl + 1) * C + col))
+                                            : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        bf16x8_to_f32(a[h], va + 8 * h);
+        bf16x8_to_f32(b[h], vb + 8 * h);
+      }
+    } else {
+      const uint8_t* xc = static_cast<const uint8_t*>(p.x);
+      const float in_ts = *p.in_ts;
+      const int gin = p.in_fmt == FMT_NV ? 16 : 32;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int64_t r = r0 + rl + q;
+        uint2 cw = make_uint2(0, 0);
+        uint32_t sa = 0;
+        if (r < R && cc < C) {
+          cw = __ldg(reinterpret_cast<const uint2*>(xc + r * (C >> 1) + (cc >> 1)));
+          sa = p.in_scales[r * (C / gin) + cc / gin];
+        }
+        const float s_a = fp4_in_scale(sa, p.in_fmt);
+        float* dst = q ? vb : va;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          dst[j] = __fmul_rn(__fmul_rn(e2m1_dec((j < 8 ? cw.x : cw.y) >> (4 * (j & 7))), s_a), in_ts);
+      }
+    }
+    const int pc = t32_col(rl);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) *reinterpret_cast<float2*>(&tile[16 * cb + j][pc]) = make_float2(va[j], vb[j]);
+  }
+  __syncthreads();
+  const uint32_t amax_in = (FMT == FMT_NV && RND != R_EDEN && RND != R_AMAX) ? *p.amax_bits : 0u;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) write_tensor_scale<FMT, RND>(p, amax_in);
+  const int orl = threadIdx.x >> 2, seg = threadIdx.x & 3;
+  const int64_t orow = c0 + orl, ocol = r0 + 32 * seg;
+  const bool active = orow < C && ocol < R;
+  float x[32];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 v = *reinterpret_cast<const float4*>(&tile[orl][t32_col(32 * seg) + 4 * i]);
+    x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+  }
+  const uint32_t acc = process32<FMT, RND, HAD>(x, active, active ? orow : 0, active ? ocol : 0, lane, p, sh, amax_in);
+  if (RND == R_AMAX || RND == R_EDEN) block_max_atomic(acc, sh, p.amax_bits, p.status);
+}
+
+// Exhaustive check of the hardware E2M1 encoder against the per-element
+// software rounding over every non-NaN fp32 bit pattern; counts mismatches.
+static __global__ void k_selftest_e2m1(unsigned long long* mismatches) {
+  unsigned long long bad = 0;
+  const uint64_t n = 1ull << 32;
+  for (uint64_t i = (uint64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < n;
+       i += uint64_t(gridDim.x) * blockDim.x * 8) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t b = uint32_t(i + j);
+      v[j] = ((b & 0x7FFFFFFFu) > 0x7F800000u) ? 0.0f : bitsf(b);   // NaN -> skip (compare 0)
+    }
+    bad += (enc8_hw(v) != enc8_sw(v)) ? 1ull : 0ull;
+  }
+  if (bad) atomicAdd(mismatches, bad);
+}
+
+}  // namespace fp4

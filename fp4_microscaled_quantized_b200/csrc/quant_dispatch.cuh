@@ -1,7 +1,7 @@
 // Host-side launch of the quantiser kernels for one loader (instantiated once
 // per loader in quant_ld*.cu so the four compile in parallel).
 #pragma once
-#include "quant_kernels.cuh"
+#include "quant_core32.cuh"
 
 namespace fp4 {
 
@@ -12,17 +12,33 @@ int num_sms();
 
 template <int LOAD, int FMT, int RND, int HAD>
 cudaError_t launch_one(const QParams& p, cudaStream_t s) {
-  if (LOAD == LD_ROW || LOAD == LD_ROW_FP4) {
+  const bool wide = (p.cols % 32) == 0;   // 32 elements per lane
+  if ((LOAD == LD_ROW || LOAD == LD_ROW_FP4) && wide) {
+    int64_t tasks = p.rows * (p.cols >> 5);
+    int64_t blocks = (tasks + 255) / 256;
+    int64_t cap = int64_t(num_sms()) * 4;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    k_quant_row32<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
+    count_launch();
+  } else if (wide) {
+    dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
+              unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
+    k_quant_trans32<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
+    count_launch();
+  } else if (LOAD == LD_ROW || LOAD == LD_ROW_FP4) {
     int64_t tasks = p.rows * (p.cols >> 3);
     int64_t blocks = (tasks + 255) / 256;
     int64_t cap = int64_t(num_sms()) * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     k_quant_row<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
+    count_launch();
   } else {
     dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
               unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
     k_quant_trans<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
+    count_launch();
   }
   return cudaGetLastError();
 }

@@ -477,6 +477,27 @@ __global__ void __launch_bounds__(256) k_eden_pass2(QParams p) {
   const float s32 = eden_tensor_scale(*p.amax_bits);
   const float inv32 = __frcp_rn(s32);
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.ts = s32;
+  if ((ng & 3) == 0) {
+    // four groups k0..k0+3 of one row per thread: one Philox block, 4-byte stores
+    for (int64_t q = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; q < (total >> 2);
+         q += int64_t(gridDim.x) * blockDim.x) {
+      const int64_t gi0 = q << 2, r = gi0 / ng, k0 = gi0 % ng;
+      const uint2 ps = *reinterpret_cast<const uint2*>(p.pseudo + gi0);
+      const uint32_t pw[4] = {ps.x & 0xFFFFu, ps.x >> 16, ps.y & 0xFFFFu, ps.y >> 16};
+      const u32x4 rb = philox_block(p.seed, uint64_t(q), TAG_SR_SCALE, p.tensor_tag);
+      const uint32_t rw[4] = {rb.x, rb.y, rb.z, rb.w};
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float S = p.eden_S[r * (p.cols / HAD) + ((k0 + j) * 16) / HAD];
+        const float t = __fmul_rn(__fmul_rn(S, bitsf(pw[j] << 16)), inv32);
+        word |= e4m3_sr(t, u24(rw[j])) << (8 * j);
+      }
+      if (p.scales) *reinterpret_cast<uint32_t*>(p.scales + gi0) = word;
+      if (p.swz) *reinterpret_cast<uint32_t*>(p.swz + swz_offset(r, k0, p.nkb)) = word;
+    }
+    return;
+  }
   for (int64_t gi = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; gi < total;
        gi += int64_t(gridDim.x) * blockDim.x) {
     int64_t r = gi / ng, k = gi % ng;

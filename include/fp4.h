@@ -81,6 +81,8 @@ typedef struct {
   uint32_t sign_tag;
 } fp4_had;
 
+/* Every pointer in fp4_qtensor except tensor_scale (4 bytes) must be 16-byte
+ * aligned; otherwise the calls return FP4_ERR_ALIGNMENT. */
 typedef struct {
   uint8_t *codes;      /* rows x cols/2, required                              */
   uint8_t *scales;     /* rows x cols/g linear; may be NULL if scales_swz set  */
@@ -156,9 +158,75 @@ int fp4_swizzle_scales(const uint8_t *scales_dev, int64_t rows, int64_t n_groups
 int fp4_gemm(const fp4_qtensor *A, const fp4_qtensor *B, void *D_dev, int32_t out_dtype,
              const uint8_t *epi_mask_dev, int32_t epi_inverse_had, fp4_stream_t stream);
 
+/* ------------------------------------------------------- linear layer --
+ * Y = X W^T forward and dX = dY W, dW = dY^T X backward, fully in FP4.
+ * X: M x K bf16, W: N x K bf16, dY: M x N bf16 (row-major, device).
+ *  FP4_RECIPE_QUARTET  [Q] Algorithm 1: MXFP4; forward H32 + QuEST (clip
+ *      masks saved); backward RHT32 + SR(3/4) on dY / dY^T / W_q^T / X_q^T,
+ *      epilogue 16/9 H32^-1( . (.) (1 - mask)).
+ *  FP4_RECIPE_QUARTET2 [QII] computation graph: NVFP4; forward RTN +
+ *      Four-Over-Six, no rotation; backward de-quantise, transpose, RHT128 on
+ *      the inner dimension, MS-EDEN; no inverse transform.
+ *  FP4_RECIPE_RTN      NVFP4 RTN on every operand, no rotation.
+ * Seeds: every random draw of one backward step is keyed by step_seed; the
+ * dX GEMM's operands share sign tag 0, the dW GEMM's sign tag 1; SR tensor
+ * tags 1 (dY), 2 (W_q^T), 3 (dY^T), 4 (X_q^T); forward tags 5 (X), 6 (W). */
+enum fp4_recipe_id { FP4_RECIPE_QUARTET = 0, FP4_RECIPE_QUARTET2 = 1, FP4_RECIPE_RTN = 2 };
+
+typedef struct {
+  int32_t fmt;            /* fp4_format of every operand                     */
+  int32_t fwd_rounding;   /* fp4_rounding of X and W                         */
+  int32_t fwd_had;        /* deterministic H block on K (0 = none)           */
+  int32_t bwd_rounding;   /* fp4_rounding of the four backward operands      */
+  int32_t bwd_had;        /* rotation block on each GEMM's inner dimension   */
+  int32_t bwd_randomized; /* 1: RHT (random signs), 0: H                     */
+  int32_t mask_epilogue;  /* 1: Quartet mask + H^-1 epilogue (fwd QuEST)     */
+  int32_t out_y, out_dx, out_dw; /* 0 fp32, 1 bf16                           */
+} fp4_recipe;
+
+/* Fill *r with a preset; returns FP4_ERR_INVALID_ARG for an unknown id. */
+int fp4_recipe_preset(int32_t id, fp4_recipe *r);
+
+/* Saved context of the forward pass, in caller-owned device memory:
+ * xq is M x K (codes, linear scales, swizzled scales, tensor scale, and the
+ * clip mask when the forward rounding is QuEST), wq is N x K likewise.
+ * Sizes: codes rows*cols/2, scales rows*cols/g, swizzled
+ * fp4_swizzled_scale_bytes(rows, cols/g), mask rows*cols/8, 4 bytes of scale. */
+typedef struct {
+  fp4_qtensor xq;
+  fp4_qtensor wq;
+} fp4_ctx;
+
+/* Device workspace bytes of fp4_linear_fwd (is_bwd = 0) or fp4_linear_bwd
+ * (is_bwd = 1): the quantiser scratch and, for the backward, the four
+ * re-quantised operands. */
+size_t fp4_linear_workspace_size(const fp4_recipe *r, int64_t M, int64_t N, int64_t K,
+                                 int32_t is_bwd);
+
+/* Forward: quantise X and W into ctx, Y_dev (M x N, r->out_y) = GEMM. */
+int fp4_linear_fwd(const void *X_dev, const void *W_dev, int64_t M, int64_t N, int64_t K,
+                   const fp4_recipe *r, uint64_t seed, void *Y_dev, fp4_ctx *ctx,
+                   void *ws_dev, size_t ws_bytes, fp4_stream_t stream);
+
+/* Backward: dX_dev (M x K, r->out_dx) and dW_dev (N x K, r->out_dw) from
+ * dY and the saved context.  Either output may be NULL to skip its GEMM. */
+int fp4_linear_bwd(const void *dY_dev, const fp4_ctx *ctx, int64_t M, int64_t N, int64_t K,
+                   const fp4_recipe *r, uint64_t step_seed, void *dX_dev, void *dW_dev,
+                   void *ws_dev, size_t ws_bytes, fp4_stream_t stream);
+
 /* Read and clear the device status word after synchronising `stream`.
  * Returns FP4_OK or the first device-side fp4_status recorded. */
 int fp4_get_last_error(fp4_stream_t stream);
+
+/* Number of CUDA kernels this library has launched since it was loaded
+ * (host-side counter, all devices and streams; no synchronisation). */
+unsigned long long fp4_launch_count(void);
+
+/* Device self-check of the E2M1 encoder: compares the hardware conversion
+ * used by the quantisers with the per-element round-to-nearest-even rounding
+ * over all 2^32 fp32 bit patterns (NaNs excluded) and ADDS the number of
+ * mismatching 8-element words to *mismatches_dev (caller zeroes it). */
+int fp4_selftest_e2m1(unsigned long long *mismatches_dev, fp4_stream_t stream);
 
 /* Static description of a status code. */
 const char *fp4_status_string(int status);

@@ -123,3 +123,30 @@ def test_empty_input_is_a_noop(cuda_lib):
     x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
     q = cuda_lib.quantize(x, qn.NVFP4, qn.MS_EDEN, 128)
     assert q.rows == 0 and cuda_lib.get_last_error() == 0
+
+
+def test_hardware_e2m1_encoder_exhaustive(cuda_lib):
+    """The hardware conversion used by the 32-per-lane path equals the
+    per-element round-to-nearest-even onto E2M1 for every fp32 input."""
+    assert cuda_lib.selftest_e2m1() == 0
+
+
+@pytest.mark.parametrize("fmt,rnd,had", [(qn.NVFP4, qn.FOUR_OVER_SIX, 0), (qn.NVFP4, qn.MS_EDEN, 16),
+                                         (qn.NVFP4, qn.SR, 16), (qn.NVFP4, qn.QUEST, 0)])
+@pytest.mark.parametrize("transpose", [False, True])
+def test_narrow_inner_dim_path(cuda_lib, fmt, rnd, had, transpose):
+    """Inner dimension 16 mod 32 runs the 8-per-lane kernels."""
+    shape = (48, 136) if transpose else (136, 48)
+    bits = syn.outlier_elements(shape, seed=9, stream=rnd)
+    g = cuda_lib.quantize(to_dev(bits), fmt, rnd, had, randomized=had > 0, seed=3, sign_tag=1,
+                          tensor_tag=2, transpose=transpose)
+    o = qn.quantize(syn.bf16_bits_to_f32(bits), fmt, rnd, had, had > 0, 3, 1, 2, transpose=transpose)
+    assert_qt_equal(g, o)
+
+
+def test_launch_counter_counts_kernels(cuda_lib):
+    x = to_dev(syn.gaussian((128, 256), 1.0, seed=1))        # no swizzle padding to zero
+    n0 = cuda_lib.launch_count()
+    cuda_lib.quantize(x, qn.NVFP4, qn.MS_EDEN, 128, randomized=True)      # pass 1 + pass 2
+    cuda_lib.quantize(x, qn.NVFP4, qn.FOUR_OVER_SIX, 0)                     # amax + quantise
+    assert cuda_lib.launch_count() - n0 == 4
