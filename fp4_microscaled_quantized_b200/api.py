@@ -176,6 +176,28 @@ def quantize(x, fmt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0, ten
     return out
 
 
+def quantize_noalloc(x, fmt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0, tensor_tag=0,
+                     transpose=False, out=None):
+    """fp4_quantize_noalloc: the same quantisation as quantize(), with the
+    library's fixed device scratch instead of a caller workspace (the C call
+    allocates nothing; only this binding allocates `out` when not given)."""
+    lib = load()
+    f = lib.fp4_quantize_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_int32, ctypes.c_int32, fp4_had, ctypes.c_uint64, ctypes.c_uint32,
+                  ctypes.POINTER(fp4_qtensor), ctypes.c_void_p]
+    in_rows, in_cols = x.shape
+    rows, cols = (in_cols, in_rows) if transpose else (in_rows, in_cols)
+    if out is None:
+        out = alloc_qtensor(rows, cols, fmt, mask=(rnd == QUEST), device=x.device)
+    cs = out.c_struct()
+    st = f(_ptr(x), in_rows, in_cols, int(transpose), fmt, rnd, GROUP[fmt],
+           fp4_had(had_block, int(randomized), sign_tag), seed, tensor_tag, ctypes.byref(cs), _stream())
+    _check(st, "fp4_quantize_noalloc")
+    return out
+
+
 def requantize(qt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0, tensor_tag=0,
                transpose=True, linear=True, swizzled=True, out=None, ws=None):
     lib = load()

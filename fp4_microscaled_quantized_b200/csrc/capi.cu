@@ -290,3 +290,45 @@ const char* fp4_status_string(int st) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- allocation-free quantise --
+// Scratch for fp4_quantize_noalloc: a fixed array in the library's own device
+// memory (every GPU that loads the library holds it until the process exits).
+// All calls share it, so two such calls that overlap on the GPU race on it.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FP4_NOALLOC_SCRATCH_BYTES];
+
+namespace fp4 {
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (with that device current) on its first use; nullptr on failure.
+static void* noalloc_scratch_ptr() {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = a;
+  }
+  return addr[dev];
+}
+}  // namespace fp4
+
+extern "C" int fp4_quantize_noalloc(const void* x, int64_t in_rows, int64_t in_cols, int32_t transpose,
+                                    int32_t fmt, int32_t rounding, int32_t group, fp4_had had, uint64_t seed,
+                                    uint32_t tensor_tag, fp4_qtensor* out, fp4_stream_t stream) {
+  if (in_rows < 0 || in_cols < 0 || (transpose != 0 && transpose != 1)) return FP4_ERR_INVALID_ARG;
+  const int64_t rows = transpose ? in_cols : in_rows, cols = transpose ? in_rows : in_cols;
+  const size_t need = fp4_quantize_workspace_size(rows, cols, fmt, rounding, had.block);
+  if (need > FP4_NOALLOC_SCRATCH_BYTES) return FP4_ERR_WORKSPACE;   // tensor too large for the array
+  void* ws = nullptr;
+  if (need > 0) {
+    ws = noalloc_scratch_ptr();
+    if (!ws) return FP4_ERR_CUDA;
+  }
+  // The same quantiser as fp4_quantize; the amax word it needs zeroed is
+  // cleared on the stream inside (cudaMemsetAsync, no allocation).
+  return fp4_quantize(x, in_rows, in_cols, transpose, fmt, rounding, group, had, seed, tensor_tag, out, ws,
+                      need, stream);
+}

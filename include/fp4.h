@@ -129,6 +129,40 @@ int fp4_quantize(const void *x_dev, int64_t in_rows, int64_t in_cols,
                  fp4_qtensor *out, void *ws_dev, size_t ws_bytes,
                  fp4_stream_t stream);
 
+/* fp4_quantize without a caller-provided workspace.  (This entry point has
+ * no counterpart in the papers; it exists for library users.)
+ *
+ * Some callers cannot allocate device memory at the moment they quantise: a
+ * host framework or serving engine that owns every byte of device memory and
+ * hands none out after start-up, a plugin that is given only its inputs and
+ * outputs, or a latency-critical loop where a cudaMalloc (which may
+ * synchronise the device) is not acceptable.  This call needs no workspace:
+ * the scratch that the global-amax and MS-EDEN modes need (amax word,
+ * pseudo-scales, EDEN factors) lives in a fixed device array of
+ * FP4_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  The call allocates and frees
+ * nothing (no cudaMalloc, no library allocator); the caller still provides x
+ * and every output buffer of `out`, exactly as for fp4_quantize, and the
+ * results are bit-identical to fp4_quantize's.
+ *  - Limit: a quantised tensor whose fp4_quantize_workspace_size exceeds
+ *    FP4_NOALLOC_SCRATCH_BYTES (4 MiB) returns FP4_ERR_WORKSPACE and launches
+ *    nothing.  That is about 26.8 million elements for MS-EDEN with 128-blocks
+ *    (16.7 million with 32-blocks, 11.1 million with 16-blocks); the other
+ *    NVFP4 modes (256 bytes) and all MXFP4 modes (none) fit at any size.
+ *  - All calls share the one array and it keeps the last call's contents; the
+ *    part that must start at zero (the amax word) is cleared on `stream`
+ *    inside the call.  Two calls whose work overlaps on the GPU (different
+ *    streams, or different host threads on one device) race on the array and
+ *    give wrong results: serialise them.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture. */
+#define FP4_NOALLOC_SCRATCH_BYTES (4u << 20)
+int fp4_quantize_noalloc(const void *x_dev, int64_t in_rows, int64_t in_cols,
+                         int32_t transpose, int32_t fmt, int32_t rounding, int32_t group,
+                         fp4_had had, uint64_t seed, uint32_t tensor_tag,
+                         fp4_qtensor *out, fp4_stream_t stream);
+
 /* Re-quantise a saved FP4 tensor [QII] computation graph backward steps 1-4:
  * de-quantise (fp32(fp32(q * s_group) * s_tensor)), optionally transpose,
  * rotate along the new inner dimension, quantise in `in->fmt` with
