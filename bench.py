@@ -16,6 +16,7 @@ step time is the max over ranks.  Prints one JSON line on rank 0.
 """
 import argparse
 import ctypes
+import hashlib
 import json
 import os
 import subprocess
@@ -409,7 +410,11 @@ def main():
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if os.path.exists(tpath):
-        traffic = json.load(open(tpath)).get("bytes_per_launch")
+        rec = json.load(open(tpath))
+        src = os.path.join(ROOT, "fp4_microscaled_quantized_b200", "csrc", "gemm_sm100.cu")
+        # counters taken on another version of the kernel do not describe this one
+        if rec.get("kernel_source_sha256") == hashlib.sha256(open(src, "rb").read()).hexdigest():
+            traffic = rec.get("bytes_per_launch")
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",

@@ -35,15 +35,6 @@ __device__ __forceinline__ uint32_t enc8_sw(const float* v) {
   return w;
 }
 
-// Grid value of an E2M1 code from its bits: magnitude m >= 2 is 2^((m>>1)-1)
-// (1 + (m&1)/2), i.e. fp32 bits (m << 22) + 0x3F000000; m = 1 is 0.5.
-__device__ __forceinline__ float e2m1_dec(uint32_t c) {
-  const uint32_t m = c & 7u;
-  uint32_t b = (m << 22) + 0x3F000000u - (m == 1u ? 0x400000u : 0u);
-  b = m ? b : 0u;
-  return bitsf(b | ((c & 8u) << 28));
-}
-
 __device__ __forceinline__ float tree16(const float* s) { return __fadd_rn(tree8(s), tree8(s + 8)); }
 __device__ __forceinline__ float tree32(const float* s) { return __fadd_rn(tree16(s), tree16(s + 16)); }
 
@@ -56,24 +47,59 @@ __device__ __forceinline__ void enc16(const float* x, float inv, bool ok, uint32
   w[1] = ok ? enc8_hw(v + 8) : 0u;
 }
 
-// fp32 squared error of 16 elements against codes * d, pairwise tree.
-__device__ __forceinline__ float sse16(const float* x, const uint32_t* w, float d) {
+// Grid magnitude of element j of a code word from the shared table (the
+// table holds the signed values by code; magnitudes are its first 8 entries).
+__device__ __forceinline__ float mag_at(const float* lut, const uint32_t* w, int j) {
+  return lut[(w[j >> 3] >> (4 * (j & 7))) & 7u];
+}
+
+// fp32 squared error of 16 elements against codes * d, pairwise tree.  The
+// code of x carries x's sign (or is 0), so x - q d = sign(x) (|x| - |q| d)
+// exactly and the square only needs magnitudes.
+__device__ __forceinline__ float sse16(const float* x, const uint32_t* w, float d, const float* lut) {
   float s[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    float e = __fsub_rn(x[j], __fmul_rn(e2m1_dec(w[j >> 3] >> (4 * (j & 7))), d));
+    float e = __fsub_rn(fabsf(x[j]), __fmul_rn(mag_at(lut, w, j), d));
     s[j] = __fmul_rn(e, e);
   }
   return tree16(s);
 }
 
-// Block FWHT over HAD consecutive elements, 32 per lane (HAD / 32 aligned
-// lanes for HAD = 128), same butterfly order as fwht8_lanes.
-template <int HAD>
-__device__ __forceinline__ void fwht32_lanes(float* x, uint32_t sign, int lane) {
+// Per-lane XOR masks that apply the randomized-Hadamard signs to loaded data
+// before it is unpacked: for bf16 pairs (sign bits 15 and 31 of each 32-bit
+// word of two elements) and for FP4 codes (bit 3 of each nibble).  `sw` holds
+// the sign bits of the lane's 32 consecutive positions.
+__device__ __forceinline__ void sign_masks_bf16(uint32_t sw, uint32_t* m16) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if ((sign >> j) & 1u) x[j] = -x[j];
+  for (int i = 0; i < 16; ++i) m16[i] = (((sw >> (2 * i)) & 1u) << 15) | (((sw >> (2 * i + 1)) & 1u) << 31);
+}
+__device__ __forceinline__ void sign_masks_fp4(uint32_t sw, uint32_t* m4) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m |= ((sw >> (8 * k + j)) & 1u) << (4 * j + 3);
+    m4[k] = m;
+  }
+}
+
+// Sign bits of the 32 consecutive positions starting at `pos` of a rotation
+// block (pos is a multiple of 32, or 0 for 16-blocks whose pattern repeats).
+template <int HAD>
+__device__ __forceinline__ uint32_t lane_signs(const Shared& sh, const QParams& p, int pos) {
+  if (HAD == 0 || !p.randomized) return 0u;
+  if (HAD == 16) return (sh.signs[0] & 0xFFFFu) | (sh.signs[0] << 16);
+  return sh.signs[(pos & (HAD - 1)) >> 5];
+}
+
+// Block FWHT over HAD consecutive elements, 32 per lane (HAD / 32 aligned
+// lanes for HAD = 128), same butterfly order as fwht8_lanes.  The random
+// signs are applied by the loaders (to the bf16 bits or the FP4 codes).  A
+// cross-lane butterfly is one fma(+-1, x, o): with the exact product by +-1 it
+// rounds exactly like x + o and o - x.
+template <int HAD>
+__device__ __forceinline__ void fwht32_lanes(float* x, int lane) {
   constexpr int HIN = HAD < 32 ? HAD : 32;
 #pragma unroll
   for (int h = 1; h < HIN; h <<= 1) {
@@ -87,11 +113,11 @@ __device__ __forceinline__ void fwht32_lanes(float* x, uint32_t sign, int lane) 
   }
 #pragma unroll
   for (int hl = 1; hl < HAD / 32; hl <<= 1) {
-    const bool upper = (lane & hl) != 0;
+    const float sgn = (lane & hl) ? -1.0f : 1.0f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       float o = __shfl_xor_sync(0xFFFFFFFFu, x[i], hl);
-      x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+      x[i] = __fmaf_rn(sgn, x[i], o);
     }
   }
   const float c = HAD == 16 ? 0.25f : (HAD == 32 ? 0.176776695296636881f : 0.0883883476483184405f);
@@ -104,18 +130,8 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
                                               const QParams& p, const Shared& sh, uint32_t amax_in) {
   constexpr int G = FMT == FMT_NV ? 16 : 32;
   constexpr int NG = 32 / G;
-  if (HAD > 0) {
-    uint32_t sign = 0;
-    if (p.randomized) {
-      if (HAD == 16) {
-        sign = sh.signs[0] & 0xFFFFu;
-        sign |= sign << 16;
-      } else {
-        sign = sh.signs[int(ocol & (HAD - 1)) >> 5];
-      }
-    }
-    fwht32_lanes<HAD>(x, sign, lane);
-  }
+  const float* lut = sh.lut;
+  if (HAD > 0) fwht32_lanes<HAD>(x, lane);      // signs already applied by the loader
   uint32_t gmb[NG];
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
@@ -153,7 +169,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
         uint32_t w6[2], w4[2];
         enc16(xg, i6, finite_pos(d6, i6), w6);
         enc16(xg, i4, finite_pos(d4, i4), w4);
-        const bool pick4 = sse16(xg, w4, d4) < sse16(xg, w6, d6);
+        const bool pick4 = sse16(xg, w4, d4, lut) < sse16(xg, w6, d6, lut);
         wg[0] = pick4 ? w4[0] : w6[0];
         wg[1] = pick4 ? w4[1] : w6[1];
         sb[g] = pick4 ? s4 : s6;
@@ -198,7 +214,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
             float d = __fmul_rn(e4m3_value(uint32_t(cc)), s32), inv = __frcp_rn(d);
             uint32_t wt[2];
             enc16(xg, inv, finite_pos(d, inv), wt);
-            float e = sse16(xg, wt, d);
+            float e = sse16(xg, wt, d, lut);
             if (e <= best) { best = e; bc = cc; }
           }
           s8 = uint32_t(bc);
@@ -226,7 +242,8 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         yy[j] = __fmul_rn(xg[j], xg[j]);
-        yq[j] = __fmul_rn(xg[j], __fmul_rn(e2m1_dec(w[2 * g + (j >> 3)] >> (4 * (j & 7))), pq));
+        // y (q p) = |y| (|q| p): the code carries y's sign (or is 0)
+        yq[j] = __fmul_rn(fabsf(xg[j]), __fmul_rn(mag_at(lut, w + 2 * g, j), pq));
       }
       num_g[g] = tree16(yy);       // the two halves of the 32-element tree
       den_g[g] = tree16(yq);
@@ -300,7 +317,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
       for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(x[j], sc);
 #pragma unroll
       for (int q = 0; q < 4; ++q) wt[q] = enc8_hw(v + 8 * q);
-      const float s = __fadd_rn(sse16(x, wt, d), sse16(x + 16, wt + 2, d));
+      const float s = __fadd_rn(sse16(x, wt, d, lut), sse16(x + 16, wt + 2, d, lut));
       if (s <= bs) { bs = s; be = e; }
       found = true;
     }
@@ -353,6 +370,13 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
   if (blockIdx.x == 0 && threadIdx.x == 0) write_tensor_scale<FMT, RND>(p, amax_in);
   uint32_t acc = 0;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  // The lane's 32 columns sit at the same offset of their rotation block on
+  // every task (cols is a multiple of the block, the stride of 32 tasks), so
+  // its sign masks are fixed for the whole loop.
+  const uint32_t sw = lane_signs<HAD>(sh, p, 32 * (lane & 3));
+  uint32_t sm[LOAD == LD_ROW ? 16 : 4];
+  if (LOAD == LD_ROW) sign_masks_bf16(sw, sm);
+  else sign_masks_fp4(sw, sm);
   for (int64_t base = int64_t(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); base < tasks; base += stride) {
     const int64_t t = base + lane;
     const bool active = t < tasks;
@@ -364,7 +388,10 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) v[i] = active ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) bf16x8_to_f32(v[i], x + 8 * i);
+      for (int i = 0; i < 4; ++i) {
+        v[i].x ^= sm[4 * i]; v[i].y ^= sm[4 * i + 1]; v[i].z ^= sm[4 * i + 2]; v[i].w ^= sm[4 * i + 3];
+        bf16x8_to_f32(v[i], x + 8 * i);
+      }
     } else {
       uint4 cw = make_uint4(0, 0, 0, 0);
       uint32_t s0 = 0, s1 = 0;
@@ -375,10 +402,10 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
         s1 = p.in_scales[orow * (p.cols / gin) + (ocol + 16) / gin];
       }
       const float sa = fp4_in_scale(s0, p.in_fmt), sbv = fp4_in_scale(s1, p.in_fmt);
-      const uint32_t cws[4] = {cw.x, cw.y, cw.z, cw.w};
+      const uint32_t cws[4] = {cw.x ^ sm[0], cw.y ^ sm[1], cw.z ^ sm[2], cw.w ^ sm[3]};
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        x[j] = __fmul_rn(__fmul_rn(e2m1_dec(cws[j >> 3] >> (4 * (j & 7))), j < 16 ? sa : sbv), in_ts);
+        x[j] = __fmul_rn(__fmul_rn(sh.lut[(cws[j >> 3] >> (4 * (j & 7))) & 15u], j < 16 ? sa : sbv), in_ts);
     }
     acc = max(acc, process32<FMT, RND, HAD>(x, active, orow, ocol, lane, p, sh, amax_in));
   }
@@ -404,7 +431,12 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
     const int rl = 64 * rh + 2 * lane;
     const int64_t cc = c0 + 16 * cb;
     float va[16], vb[16];
+    // Input rows rl and rl + 1 are positions rl, rl + 1 of their rotation
+    // block along the output rows (r0 is a multiple of 128): one sign each.
+    const uint32_t sgn_a = (lane_signs<HAD>(sh, p, rl) >> (rl & 31)) & 1u;
+    const uint32_t sgn_b = (lane_signs<HAD>(sh, p, rl + 1) >> ((rl + 1) & 31)) & 1u;
     if (LOAD == LD_TRANS) {
+      const uint32_t ma = sgn_a * 0x80008000u, mb = sgn_b * 0x80008000u;
       const uint16_t* xb = static_cast<const uint16_t*>(p.x);
       uint4 a[2], b[2];
 #pragma unroll
@@ -417,6 +449,8 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+        a[h].x ^= ma; a[h].y ^= ma; a[h].z ^= ma; a[h].w ^= ma;
+        b[h].x ^= mb; b[h].y ^= mb; b[h].z ^= mb; b[h].w ^= mb;
         bf16x8_to_f32(a[h], va + 8 * h);
         bf16x8_to_f32(b[h], vb + 8 * h);
       }
@@ -433,11 +467,13 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
           cw = __ldg(reinterpret_cast<const uint2*>(xc + r * (C >> 1) + (cc >> 1)));
           sa = p.in_scales[r * (C / gin) + cc / gin];
         }
+        const uint32_t m = (q ? sgn_b : sgn_a) * 0x88888888u;
+        cw.x ^= m; cw.y ^= m;
         const float s_a = fp4_in_scale(sa, p.in_fmt);
         float* dst = q ? vb : va;
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          dst[j] = __fmul_rn(__fmul_rn(e2m1_dec((j < 8 ? cw.x : cw.y) >> (4 * (j & 7))), s_a), in_ts);
+          dst[j] = __fmul_rn(__fmul_rn(sh.lut[((j < 8 ? cw.x : cw.y) >> (4 * (j & 7))) & 15u], s_a), in_ts);
       }
     }
     const int pc = t32_col(rl);
