@@ -411,9 +411,9 @@ def main():
     tpath = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if os.path.exists(tpath):
         rec = json.load(open(tpath))
-        src = os.path.join(ROOT, "fp4_microscaled_quantized_b200", "csrc", "gemm_sm100.cu")
+        gemm_src = os.path.join(ROOT, "fp4_microscaled_quantized_b200", "csrc", "gemm_sm100.cu")
         # counters taken on another version of the kernel do not describe this one
-        if rec.get("kernel_source_sha256") == hashlib.sha256(open(src, "rb").read()).hexdigest():
+        if rec.get("kernel_source_sha256") == hashlib.sha256(open(gemm_src, "rb").read()).hexdigest():
             traffic = rec.get("bytes_per_launch")
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

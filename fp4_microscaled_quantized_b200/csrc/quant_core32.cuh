@@ -6,6 +6,7 @@
 // 8-per-lane path in quant_kernels.cuh (same butterfly order, same pairwise
 // trees), so both produce identical bits.
 #pragma once
+#include <cuda_fp16.h>
 #include "quant_kernels.cuh"
 
 namespace fp4 {
@@ -38,32 +39,91 @@ __device__ __forceinline__ uint32_t enc8_sw(const float* v) {
 __device__ __forceinline__ float tree16(const float* s) { return __fadd_rn(tree8(s), tree8(s + 8)); }
 __device__ __forceinline__ float tree32(const float* s) { return __fadd_rn(tree16(s), tree16(s + 16)); }
 
+// Packed fp32 pair arithmetic (two independent IEEE round-to-nearest results
+// per instruction).  a - b is fma(b, -1, a): the product is exact, so it
+// rounds exactly like the subtraction, signed zeros included.
+__device__ __forceinline__ float2 ld2(const float* x, int i) { return make_float2(x[i], x[i + 1]); }
+__device__ __forceinline__ void st2(float* x, int i, float2 v) { x[i] = v.x; x[i + 1] = v.y; }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// The same value as tree16 (level 0 adds (2i, 2i+1), then pairs of pairs),
+// with the upper levels packed: level-0 sums are paired as (n_i, n_{i+4}), so
+// levels 1 and 2 each add two tree nodes per instruction.
+__device__ __forceinline__ float tree16p(const float* s) {
+  const float2 a0 = make_float2(__fadd_rn(s[0], s[1]), __fadd_rn(s[8], s[9]));
+  const float2 a1 = make_float2(__fadd_rn(s[2], s[3]), __fadd_rn(s[10], s[11]));
+  const float2 a2 = make_float2(__fadd_rn(s[4], s[5]), __fadd_rn(s[12], s[13]));
+  const float2 a3 = make_float2(__fadd_rn(s[6], s[7]), __fadd_rn(s[14], s[15]));
+  const float2 c = __fadd2_rn(__fadd2_rn(a0, a1), __fadd2_rn(a2, a3));
+  return __fadd_rn(c.x, c.y);
+}
+
+// Three-input maximum that propagates NaN (so a non-finite input is seen by
+// the status check); on finite inputs it is the exact maximum.
+__device__ __forceinline__ float max3n(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Bits of max |x| over 16 consecutive values.  Absolute values are
+// non-negative, so the float maximum and the maximum of the bit patterns
+// agree.
+__device__ __forceinline__ uint32_t absmax16(const float* x) {
+  const float a0 = max3n(fabsf(x[0]), fabsf(x[1]), fabsf(x[2]));
+  const float a1 = max3n(fabsf(x[3]), fabsf(x[4]), fabsf(x[5]));
+  const float a2 = max3n(fabsf(x[6]), fabsf(x[7]), fabsf(x[8]));
+  const float a3 = max3n(fabsf(x[9]), fabsf(x[10]), fabsf(x[11]));
+  const float a4 = max3n(fabsf(x[12]), fabsf(x[13]), fabsf(x[14]));
+  const float b0 = max3n(a0, a1, a2), b1 = max3n(a3, a4, fabsf(x[15]));
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(b0), "f"(b1));
+  return fbits(r);
+}
+
 // 16 codes of x * inv (or zeros when !ok) into two words.
 __device__ __forceinline__ void enc16(const float* x, float inv, bool ok, uint32_t* w) {
   float v[16];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(x[j], inv);
+  for (int j = 0; j < 16; j += 2) st2(v, j, __fmul2_rn(ld2(x, j), splat2(inv)));
   w[0] = ok ? enc8_hw(v) : 0u;
   w[1] = ok ? enc8_hw(v + 8) : 0u;
 }
 
-// Grid magnitude of element j of a code word from the shared table (the
-// table holds the signed values by code; magnitudes are its first 8 entries).
-__device__ __forceinline__ float mag_at(const float* lut, const uint32_t* w, int j) {
-  return lut[(w[j >> 3] >> (4 * (j & 7))) & 7u];
+// Signed grid values of the 8 codes of a word (element j from bits 4j..4j+3):
+// the packed E2M1 -> f16x2 conversion, then f16 -> f32, both exact.  Code 8
+// gives -0.
+__device__ __forceinline__ void dec8(uint32_t w, float* q) {
+  uint32_t h[4];
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[k]));
+    q[2 * k] = f.x;
+    q[2 * k + 1] = f.y;
+  }
 }
 
-// fp32 squared error of 16 elements against codes * d, pairwise tree.  The
-// code of x carries x's sign (or is 0), so x - q d = sign(x) (|x| - |q| d)
-// exactly and the square only needs magnitudes.
-__device__ __forceinline__ float sse16(const float* x, const uint32_t* w, float d, const float* lut) {
-  float s[16];
+// fp32 squared error of 16 elements against codes * d, pairwise tree:
+// e = x - fp32(q d), s = fp32(e e).
+__device__ __forceinline__ float sse16(const float* x, const uint32_t* w, float d) {
+  float q[16], s[16];
+  dec8(w[0], q);
+  dec8(w[1], q + 8);
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    float e = __fsub_rn(fabsf(x[j]), __fmul_rn(mag_at(lut, w, j), d));
-    s[j] = __fmul_rn(e, e);
+  for (int j = 0; j < 16; j += 2) {
+    const float2 e = sub2(ld2(x, j), __fmul2_rn(ld2(q, j), splat2(d)));
+    st2(s, j, __fmul2_rn(e, e));
   }
-  return tree16(s);
+  return tree16p(s);
 }
 
 // Per-lane XOR masks that apply the randomized-Hadamard signs to loaded data
@@ -95,34 +155,41 @@ __device__ __forceinline__ uint32_t lane_signs(const Shared& sh, const QParams& 
 
 // Block FWHT over HAD consecutive elements, 32 per lane (HAD / 32 aligned
 // lanes for HAD = 128), same butterfly order as fwht8_lanes.  The random
-// signs are applied by the loaders (to the bf16 bits or the FP4 codes).  A
-// cross-lane butterfly is one fma(+-1, x, o): with the exact product by +-1 it
-// rounds exactly like x + o and o - x.
+// signs are applied by the loaders (to the bf16 bits or the FP4 codes).  The
+// h = 1 stage works inside the natural pairs (2i, 2i+1); every later stage,
+// the cross-lane ones (x + o on the lower lane, o - x on the upper: one
+// fma(+-1, x, o)) and the final scaling run two elements per instruction.
 template <int HAD>
 __device__ __forceinline__ void fwht32_lanes(float* x, int lane) {
   constexpr int HIN = HAD < 32 ? HAD : 32;
 #pragma unroll
-  for (int h = 1; h < HIN; h <<= 1) {
+  for (int i = 0; i < 32; i += 2) {
+    const float a = x[i], b = x[i + 1];
+    x[i] = __fadd_rn(a, b);
+    x[i + 1] = __fsub_rn(a, b);
+  }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+  for (int h = 2; h < HIN; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
       if (i & h) continue;
-      float a = x[i], b = x[i + h];
-      x[i] = __fadd_rn(a, b);
-      x[i + h] = __fsub_rn(a, b);
+      const float2 a = ld2(x, i), b = ld2(x, i + h);
+      st2(x, i, __fadd2_rn(a, b));
+      st2(x, i + h, sub2(a, b));
     }
   }
 #pragma unroll
   for (int hl = 1; hl < HAD / 32; hl <<= 1) {
-    const float sgn = (lane & hl) ? -1.0f : 1.0f;
+    const float2 sgn = splat2((lane & hl) ? -1.0f : 1.0f);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float o = __shfl_xor_sync(0xFFFFFFFFu, x[i], hl);
-      x[i] = __fmaf_rn(sgn, x[i], o);
+    for (int i = 0; i < 32; i += 2) {
+      const float2 o = make_float2(__shfl_xor_sync(0xFFFFFFFFu, x[i], hl), __shfl_xor_sync(0xFFFFFFFFu, x[i + 1], hl));
+      st2(x, i, __ffma2_rn(sgn, ld2(x, i), o));
     }
   }
   const float c = HAD == 16 ? 0.25f : (HAD == 32 ? 0.176776695296636881f : 0.0883883476483184405f);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) x[j] = __fmul_rn(x[j], c);
+  for (int j = 0; j < 32; j += 2) st2(x, j, __fmul2_rn(ld2(x, j), splat2(c)));
 }
 
 template <int FMT, int RND, int HAD>
@@ -130,15 +197,13 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
                                               const QParams& p, const Shared& sh, uint32_t amax_in) {
   constexpr int G = FMT == FMT_NV ? 16 : 32;
   constexpr int NG = 32 / G;
-  const float* lut = sh.lut;
   if (HAD > 0) fwht32_lanes<HAD>(x, lane);      // signs already applied by the loader
   uint32_t gmb[NG];
-#pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    uint32_t m = 0;
-#pragma unroll
-    for (int j = 0; j < G; ++j) m = max(m, absbits(x[g * G + j]));
-    gmb[g] = m;
+  if (NG == 2) {
+    gmb[0] = absmax16(x);
+    gmb[NG - 1] = absmax16(x + 16);
+  } else {
+    gmb[0] = max(absmax16(x), absmax16(x + 16));
   }
   uint32_t lmax = NG == 2 ? max(gmb[0], gmb[NG - 1]) : gmb[0];
   if (!active) lmax = 0;
@@ -169,7 +234,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
         uint32_t w6[2], w4[2];
         enc16(xg, i6, finite_pos(d6, i6), w6);
         enc16(xg, i4, finite_pos(d4, i4), w4);
-        const bool pick4 = sse16(xg, w4, d4, lut) < sse16(xg, w6, d6, lut);
+        const bool pick4 = sse16(xg, w4, d4) < sse16(xg, w6, d6);
         wg[0] = pick4 ? w4[0] : w6[0];
         wg[1] = pick4 ? w4[1] : w6[1];
         sb[g] = pick4 ? s4 : s6;
@@ -214,7 +279,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
             float d = __fmul_rn(e4m3_value(uint32_t(cc)), s32), inv = __frcp_rn(d);
             uint32_t wt[2];
             enc16(xg, inv, finite_pos(d, inv), wt);
-            float e = sse16(xg, wt, d, lut);
+            float e = sse16(xg, wt, d);
             if (e <= best) { best = e; bc = cc; }
           }
           s8 = uint32_t(bc);
@@ -238,15 +303,17 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
       const float pq = e8m3_round(__fdiv_rn(bitsf(gmb[g]), FP4_EDEN_S));
       const float inv = __frcp_rn(pq);
       enc16(xg, inv, finite_pos(pq, inv), w + 2 * g);
-      float yy[16], yq[16];
+      float q[16], yy[16], yq[16];
+      dec8(w[2 * g], q);
+      dec8(w[2 * g + 1], q + 8);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        yy[j] = __fmul_rn(xg[j], xg[j]);
-        // y (q p) = |y| (|q| p): the code carries y's sign (or is 0)
-        yq[j] = __fmul_rn(fabsf(xg[j]), __fmul_rn(mag_at(lut, w + 2 * g, j), pq));
+      for (int j = 0; j < 16; j += 2) {
+        const float2 y2 = ld2(xg, j);
+        st2(yy, j, __fmul2_rn(y2, y2));
+        st2(yq, j, __fmul2_rn(y2, __fmul2_rn(ld2(q, j), splat2(pq))));
       }
-      num_g[g] = tree16(yy);       // the two halves of the 32-element tree
-      den_g[g] = tree16(yq);
+      num_g[g] = tree16p(yy);      // the two halves of the 32-element tree
+      den_g[g] = tree16p(yq);
       sb[g] = fbits(pq) >> 16;     // bf16 pseudo-scale (exact)
     }
     if (active) {
@@ -273,7 +340,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
     if (RND == R_RTN) {
       float v[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(x[j], sc);
+      for (int j = 0; j < 32; j += 2) st2(v, j, __fmul2_rn(ld2(x, j), splat2(sc)));
 #pragma unroll
       for (int k = 0; k < 4; ++k) w[k] = enc8_hw(v + 8 * k);
     } else {
@@ -317,7 +384,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
       for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(x[j], sc);
 #pragma unroll
       for (int q = 0; q < 4; ++q) wt[q] = enc8_hw(v + 8 * q);
-      const float s = __fadd_rn(sse16(x, wt, d, lut), sse16(x + 16, wt + 2, d, lut));
+      const float s = __fadd_rn(sse16(x, wt, d), sse16(x + 16, wt + 2, d));
       if (s <= bs) { bs = s; be = e; }
       found = true;
     }
@@ -404,8 +471,10 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
       const float sa = fp4_in_scale(s0, p.in_fmt), sbv = fp4_in_scale(s1, p.in_fmt);
       const uint32_t cws[4] = {cw.x ^ sm[0], cw.y ^ sm[1], cw.z ^ sm[2], cw.w ^ sm[3]};
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        x[j] = __fmul_rn(__fmul_rn(sh.lut[(cws[j >> 3] >> (4 * (j & 7))) & 15u], j < 16 ? sa : sbv), in_ts);
+      for (int k = 0; k < 4; ++k) dec8(cws[k], x + 8 * k);
+#pragma unroll
+      for (int j = 0; j < 32; j += 2)
+        st2(x, j, __fmul2_rn(__fmul2_rn(ld2(x, j), splat2(j < 16 ? sa : sbv)), splat2(in_ts)));
     }
     acc = max(acc, process32<FMT, RND, HAD>(x, active, orow, ocol, lane, p, sh, amax_in));
   }
@@ -468,12 +537,12 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
           sa = p.in_scales[r * (C / gin) + cc / gin];
         }
         const uint32_t m = (q ? sgn_b : sgn_a) * 0x88888888u;
-        cw.x ^= m; cw.y ^= m;
         const float s_a = fp4_in_scale(sa, p.in_fmt);
         float* dst = q ? vb : va;
+        dec8(cw.x ^ m, dst);
+        dec8(cw.y ^ m, dst + 8);
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          dst[j] = __fmul_rn(__fmul_rn(sh.lut[((j < 8 ? cw.x : cw.y) >> (4 * (j & 7))) & 15u], s_a), in_ts);
+        for (int j = 0; j < 16; j += 2) st2(dst, j, __fmul2_rn(__fmul2_rn(ld2(dst, j), splat2(s_a)), splat2(in_ts)));
       }
     }
     const int pc = t32_col(rl);
@@ -497,7 +566,8 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
 }
 
 // Exhaustive check of the hardware E2M1 encoder against the per-element
-// software rounding over every non-NaN fp32 bit pattern; counts mismatches.
+// software rounding over every non-NaN fp32 bit pattern, and of the hardware
+// decoder over every byte of two codes; counts mismatches.
 static __global__ void k_selftest_e2m1(unsigned long long* mismatches) {
   unsigned long long bad = 0;
   const uint64_t n = 1ull << 32;
@@ -510,6 +580,15 @@ static __global__ void k_selftest_e2m1(unsigned long long* mismatches) {
       v[j] = ((b & 0x7FFFFFFFu) > 0x7F800000u) ? 0.0f : bitsf(b);   // NaN -> skip (compare 0)
     }
     bad += (enc8_hw(v) != enc8_sw(v)) ? 1ull : 0ull;
+  }
+  // The hardware decoder against the code table, over every pair of codes.
+  if (blockIdx.x == 0) {
+    for (uint32_t c = threadIdx.x; c < 256u; c += blockDim.x) {
+      float q[8];
+      dec8(c | (c << 8) | (c << 16) | (c << 24), q);
+      for (int j = 0; j < 8; ++j)
+        bad += (fbits(q[j]) != fbits(e2m1_value((c >> (4 * (j & 1))) & 15u))) ? 1ull : 0ull;
+    }
   }
   if (bad) atomicAdd(mismatches, bad);
 }

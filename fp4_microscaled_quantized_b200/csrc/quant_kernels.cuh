@@ -108,7 +108,6 @@ __device__ __forceinline__ void encode_rtn8(const float* x, float inv, bool ok, 
 struct Shared {
   uint32_t signs[4];   // RHT sign bits of one rotation block (<= 128)
   uint32_t red[32];    // block reductions
-  float lut[16];       // E2M1 code -> grid value (signed), for table decoding
 };
 
 // ------------------------------------------------------------------ core --
@@ -314,7 +313,6 @@ __device__ __forceinline__ uint32_t process8(float* x, bool active, int64_t orow
 template <int HAD>
 __device__ __forceinline__ void load_signs(Shared& sh, const QParams& p) {
   if (threadIdx.x < 4) sh.signs[threadIdx.x] = 0;
-  if (threadIdx.x < 16) sh.lut[threadIdx.x] = e2m1_value(threadIdx.x);
   __syncthreads();
   if (HAD > 0 && p.randomized && threadIdx.x < HAD / 4) {
     u32x4 b = philox_block(p.seed, threadIdx.x, TAG_RHT_SIGN, p.sign_tag);

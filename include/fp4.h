@@ -256,10 +256,12 @@ int fp4_get_last_error(fp4_stream_t stream);
  * (host-side counter, all devices and streams; no synchronisation). */
 unsigned long long fp4_launch_count(void);
 
-/* Device self-check of the E2M1 encoder: compares the hardware conversion
+/* Device self-check of the E2M1 conversions: compares the hardware encoder
  * used by the quantisers with the per-element round-to-nearest-even rounding
- * over all 2^32 fp32 bit patterns (NaNs excluded) and ADDS the number of
- * mismatching 8-element words to *mismatches_dev (caller zeroes it). */
+ * over all 2^32 fp32 bit patterns (NaNs excluded), and the hardware decoder
+ * (E2M1 pair -> f16x2 -> fp32) with the code table over all 256 code pairs.
+ * ADDS the number of mismatching encoded words plus mismatching decoded
+ * values to *mismatches_dev (caller zeroes it). */
 int fp4_selftest_e2m1(unsigned long long *mismatches_dev, fp4_stream_t stream);
 
 /* Static description of a status code. */
