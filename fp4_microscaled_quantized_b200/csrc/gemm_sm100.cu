@@ -19,6 +19,7 @@
 // Every mbarrier wait is bounded; on timeout the kernel records
 // FP4_ERR_TIMEOUT, stops issuing work, frees its TMEM and returns.
 #include <cuda.h>
+#include <cstdlib>
 #include <mutex>
 
 #include "../../include/fp4.h"
@@ -42,9 +43,10 @@ constexpr int STG_BYTES = BM * 128;                  // epilogue staging: 128 ro
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * STG_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int THREADS = 384;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns: the accumulator, then two scale-factor buffers (SFA 16 + SFB
-// 32 columns each) so the stagers fill one while the MMAs read the other.
+// TMEM columns: the accumulator, then NSF scale-factor buffers (SFA 16 + SFB
+// 32 columns each) so the stagers run ahead of the MMAs.
 constexpr uint32_t ACC_COL = 0, SF_COL = 256, SF_BUF_COLS = 48, SFB_OFF = 16;
+constexpr int NSF = 4;                               // scale-factor TMEM buffers (256 + 4 x 48 <= 512 columns)
 constexpr unsigned long long WAIT_LIMIT = 4000000000ull;  // ~2 s of SM clocks
 
 enum : int { OUT_F32 = 0, OUT_BF16 = 1 };
@@ -243,8 +245,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* sf_full = acc_empty + 1;
-  uint64_t* sf_empty = sf_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + 2);
+  uint64_t* sf_empty = sf_full + NSF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_empty + NSF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -256,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 128);
-    for (int b = 0; b < 2; ++b) { mbar_init(&sf_full[b], 128); mbar_init(&sf_empty[b], 1); }
+    for (int b = 0; b < NSF; ++b) { mbar_init(&sf_full[b], 128); mbar_init(&sf_empty[b], 1); }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -302,14 +304,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     // i % STAGES and scale buffer i % 2.
     int s = 0, buf = 0;
     uint32_t ph = 0, acc_ph = 0;
-    int use[2] = {0, 0};
+    uint32_t sph = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok && t < ntiles && !*abort_flag; t += gridDim.x) {
       if (!mbar_wait(acc_empty, acc_ph ^ 1, abort_flag, p.status)) break;
       tc_fence_after();
       for (int64_t kt = 0; kt < nkt; ++kt) {
         if (!mbar_wait(&full[s], ph, abort_flag, p.status)) { ok = false; break; }
-        if (!mbar_wait(&sf_full[buf], uint32_t(use[buf] & 1), abort_flag, p.status)) { ok = false; break; }
+        if (!mbar_wait(&sf_full[buf], sph, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
         const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
         const int n_mma = kel / 64;
@@ -326,8 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_commit(&empty[s]);
         tc_commit(&sf_empty[buf]);
         if (kt == nkt - 1) tc_commit(acc_full);
-        ++use[buf];
-        buf ^= 1;
+        if (++buf == NSF) { buf = 0; sph ^= 1; }
         if (++s == STAGES) { s = 0; ph ^= 1; }
       }
       acc_ph ^= 1;
@@ -340,11 +341,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;
     int s = 0, buf = 0;
     uint32_t ph = 0;
-    int use[2] = {0, 0};
+    uint32_t sph = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
       for (int64_t kt = 0; kt < nkt; ++kt) {
-        const bool a = mbar_wait(&sf_empty[buf], uint32_t(use[buf] & 1) ^ 1u, abort_flag, p.status);
+        const bool a = mbar_wait(&sf_empty[buf], sph ^ 1u, abort_flag, p.status);
         const bool b = a && mbar_wait(&full[s], ph, abort_flag, p.status);
         if (__any_sync(0xFFFFFFFFu, !b)) { ok = false; break; }
         tc_fence_after();
@@ -377,8 +378,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         mbar_arrive(&sf_full[buf]);
-        ++use[buf];
-        buf ^= 1;
+        if (++buf == NSF) { buf = 0; sph ^= 1; }
         if (++s == STAGES) { s = 0; ph ^= 1; }
       }
     }
@@ -476,6 +476,405 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+// ------------------------------------------------- CTA-pair (2-SM) kernel --
+// The same GEMM on 256 x 256 output tiles computed by a cluster of two CTAs
+// with cta_group::2 MMAs: CTA r of the pair loads rows r*128.. of the tile's A
+// rows and of its B rows, the leader (rank 0) issues MMAs with M = 256 that
+// read both CTAs' shared memory, and each CTA keeps its 128 x 256 half of the
+// accumulator in its own tensor memory.  Each CTA thus moves half the B
+// bytes per MMA of the one-CTA kernel, which buys two more pipeline stages.
+//   operands: both CTAs' TMA loads complete on the leader's full[s]
+//             (expected bytes set by the leader's producer);
+//   scales:   each CTA loads its own scale atoms (its 128 A rows, all 256 B
+//             rows) and its stagers write its own TMEM, then arrive on the
+//             leader's sf_full[b];
+//   releases: the leader's commits arrive on empty[s], sf_empty[b] and
+//             acc_full in both CTAs (tcgen05.commit multicast);
+//   epilogue: each CTA drains its half and arrives on the leader's acc_empty.
+namespace pair {
+
+constexpr int STAGES = 5;
+constexpr int A_BYTES = 128 * 128;                   // this CTA's 128 A rows x 128 bytes
+constexpr int B_BYTES = 128 * 128;                   // this CTA's 128 B rows
+constexpr int SFA_BYTES = 4 * 512;
+constexpr int SFB_BYTES = 8 * 512;                   // both 128-row blocks of the tile's B
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * STG_BYTES + 1024 + 256;
+static_assert(SMEM_BYTES <= 232448, "shared memory of the CTA-pair kernel");
+
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Shared::cluster address of the same object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// Arrive on a barrier of either CTA of the pair (default .release.cta
+// semantics: the data it orders is tensor-memory state, ordered by the
+// tcgen05 fences around the arrive and the wait).
+__device__ __forceinline__ void arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ bool try_c(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false and the abort flag raised when the limit is hit.
+__device__ __forceinline__ bool wait_c(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status) {
+  if (try_c(b, parity)) return true;
+  const unsigned long long t0 = clock64();
+  while (true) {
+    if (try_c(b, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > WAIT_LIMIT) {
+      *abort_flag = 1;
+      flag_status(status, ST_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// TMA tile load whose completion is counted on the leader CTA's barrier (the
+// barrier address with the peer bit cleared).
+__device__ __forceinline__ void tma_load_pair(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar) & 0xFEFFFFFFu)
+      : "memory");
+}
+
+__device__ __forceinline__ void commit_both(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void commit_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int FMT>
+__device__ __forceinline__ void mma_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, uint32_t acc) {
+  if (FMT == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+        : "memory");
+  }
+}
+
+// Pair tile order: groups of 8 256-row blocks sweep all 256-column blocks.
+__device__ __forceinline__ void tile_coords2(int64_t t, int64_t nm, int64_t nn, int64_t& mb, int64_t& nb) {
+  const int64_t G = 8;
+  int64_t per_group = G * nn;
+  int64_t g = t / per_group, r = t % per_group;
+  int64_t gm = nm - g * G < G ? nm - g * G : G;
+  mb = g * G + r % gm;
+  nb = r / gm;
+}
+
+template <int FMT, int OUT, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                const __grid_constant__ CUtensorMap map_d, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * A_BYTES;
+  uint8_t* sSFA = sB + STAGES * B_BYTES;
+  uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
+  uint8_t* sStage = sSFB + STAGES * SFB_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sStage + 2 * STG_BYTES);   // leader: operand bytes of both CTAs
+  uint64_t* empty = full + STAGES;                                          // both: slot consumed by the MMAs
+  uint64_t* sf_ld = empty + STAGES;                                         // both: this CTA's scale atoms landed
+  uint64_t* acc_full = sf_ld + STAGES;                                      // both
+  uint64_t* acc_empty = acc_full + 1;                                       // leader: 4 warps x 2 CTAs
+  uint64_t* sf_full = acc_empty + 1;                                        // leader: 4 warps x 2 CTAs (x NSF)
+  uint64_t* sf_empty = sf_full + NSF;                                       // both
+  uint64_t* drain = sf_empty + NSF;                                         // leader: MMAs retired
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cta_rank();
+  const bool leader = rank == 0;
+  const int64_t nm = (p.M + 255) / 256, nn = (p.N + BN - 1) / BN, ntiles = nm * nn;
+  const int64_t nkt = (p.K + BK - 1) / BK;
+  const int64_t pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  constexpr int G = FMT == 1 ? 16 : 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_ld[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);
+    for (int b = 0; b < NSF; ++b) { mbar_init(&sf_full[b], 8); mbar_init(&sf_empty[b], 1); }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();                                   // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // the leader's barriers that both CTAs arrive on
+  const uint32_t acc_empty_l = mapa(acc_empty, 0);
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------ TMA producer --
+    int s = 0;
+    uint32_t ph = 0;
+    const int64_t nrb_a = (p.M + 127) / 128, nrb_b = (p.N + 127) / 128;
+    for (int64_t t = pair_id; t < ntiles && !*abort_flag; t += npairs) {
+      int64_t mb, nb;
+      tile_coords2(t, nm, nn, mb, nb);
+      const int64_t ra = mb * 2 + rank, rb = nb * 2 + rank;          // this CTA's 128-row blocks
+      // 128-row halves that exist (a half entirely past M or N is not loaded)
+      const int a_halves = (mb * 2 + 1 < nrb_a) ? 2 : 1, b_halves = (nb * 2 + 1 < nrb_b) ? 2 : 1;
+      const bool load_a = ra < nrb_a, load_b = rb < nrb_b;
+      for (int64_t kt = 0; kt < nkt; ++kt) {
+        if (!wait_c(&empty[s], ph ^ 1, abort_flag, p.status)) break;
+        const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
+        const int n_mma = kel / 64;
+        const int atoms = FMT == 1 ? n_mma : (n_mma + 1) / 2;
+        const int64_t atom0 = kt * (BK / G / 4);
+        if (leader) mbar_expect_tx(&full[s], uint32_t((a_halves + b_halves) * A_BYTES));
+        if (load_a) tma_load_pair(sA + s * A_BYTES, &map_a, int(kt * (BK / 2)), int(ra * 128), &full[s]);
+        if (load_b) tma_load_pair(sB + s * B_BYTES, &map_b, int(kt * (BK / 2)), int(rb * 128), &full[s]);
+        const uint32_t sf_bytes = uint32_t(atoms) * 512u * uint32_t((load_a ? 1 : 0) + b_halves);
+        mbar_expect_tx(&sf_ld[s], sf_bytes);
+        if (load_a) bulk_load(sSFA + s * SFA_BYTES, p.sfa + (ra * p.nkb + atom0) * 512, atoms * 512u, &sf_ld[s]);
+        for (int r = 0; r < b_halves; ++r)
+          bulk_load(sSFB + s * SFB_BYTES + r * 4 * 512, p.sfb + ((nb * 2 + r) * p.nkb + atom0) * 512,
+                    atoms * 512u, &sf_ld[s]);
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+    }
+    if (*abort_flag) {                               // let copies already issued land before teardown
+      const unsigned long long t0 = clock64();
+      while (clock64() - t0 < 4000000ull) {}
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // --------------------------------------------------------- MMA issue --
+    int s = 0, buf = 0;
+    uint32_t ph = 0, acc_ph = 0;
+    uint32_t sph = 0;
+    bool ok = true, issued = false;
+    for (int64_t t = pair_id; ok && t < ntiles && !*abort_flag; t += npairs) {
+      if (!wait_c(acc_empty, acc_ph ^ 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      for (int64_t kt = 0; kt < nkt; ++kt) {
+        if (!wait_c(&full[s], ph, abort_flag, p.status)) { ok = false; break; }
+        if (!wait_c(&sf_full[buf], sph, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
+        const int n_mma = kel / 64;
+        const uint32_t a_base = smem_u32(sA + s * A_BYTES), b_base = smem_u32(sB + s * B_BYTES);
+        const uint32_t sfbase = tmem + SF_COL + SF_BUF_COLS * uint32_t(buf);
+        for (int kk = 0; kk < n_mma; ++kk) {
+          const int atom = FMT == 1 ? kk : kk / 2;
+          const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
+          const uint32_t sfa = (sfbase + 4 * atom) | (sf_id << 30);
+          const uint32_t sfb = (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30);
+          mma_pair<FMT>(tmem + ACC_COL, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
+                        idesc(FMT, BN, 256, sf_id, sf_id), sfa, sfb, (kt > 0 || kk > 0) ? 1u : 0u);
+        }
+        issued = true;
+        commit_both(&empty[s]);
+        commit_both(&sf_empty[buf]);
+        if (kt == nkt - 1) commit_both(acc_full);
+        if (++buf == NSF) { buf = 0; sph ^= 1; }
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+      acc_ph ^= 1;
+    }
+    if (issued) {                                    // every MMA retired before teardown
+      commit_local(drain);                           // (bounded, and also after an abort)
+      const unsigned long long t0 = clock64();
+      while (!try_c(drain, 0) && clock64() - t0 < WAIT_LIMIT) {}
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------- scale factors -> TMEM --
+    const int q = warp & 3;
+    int s = 0, buf = 0;
+    uint32_t ph = 0;
+    uint32_t sph = 0;
+    bool ok = true;
+    for (int64_t t = pair_id; ok && t < ntiles; t += npairs) {
+      for (int64_t kt = 0; kt < nkt; ++kt) {
+        const bool a = wait_c(&sf_empty[buf], sph ^ 1u, abort_flag, p.status);
+        const bool b = a && wait_c(&sf_ld[s], ph, abort_flag, p.status);
+        if (__any_sync(0xFFFFFFFFu, !b)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t va[16], vb[32];
+        const uint8_t* sa = sSFA + s * SFA_BYTES + lane * 16;
+        const uint8_t* sb = sSFB + s * SFB_BYTES + lane * 16;
+#pragma unroll
+        for (int at = 0; at < 4; ++at) {
+          const uint4 x = *reinterpret_cast<const uint4*>(sa + at * 512);
+          va[4 * at] = x.x; va[4 * at + 1] = x.y; va[4 * at + 2] = x.z; va[4 * at + 3] = x.w;
+#pragma unroll
+          for (int rbk = 0; rbk < 2; ++rbk) {
+            const uint4 y = *reinterpret_cast<const uint4*>(sb + (rbk * 4 + at) * 512);
+            const int o = 8 * at + 4 * rbk;
+            vb[o] = y.x; vb[o + 1] = y.y; vb[o + 2] = y.z; vb[o + 3] = y.w;
+          }
+        }
+        const uint32_t base = tmem + (uint32_t(q * 32) << 16) + SF_COL + SF_BUF_COLS * uint32_t(buf);
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(base),
+            "r"(va[0]), "r"(va[1]), "r"(va[2]), "r"(va[3]), "r"(va[4]), "r"(va[5]), "r"(va[6]), "r"(va[7]), "r"(va[8]),
+            "r"(va[9]), "r"(va[10]), "r"(va[11]), "r"(va[12]), "r"(va[13]), "r"(va[14]), "r"(va[15]));
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+            "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(base + SFB_OFF),
+            "r"(vb[0]), "r"(vb[1]), "r"(vb[2]), "r"(vb[3]), "r"(vb[4]), "r"(vb[5]), "r"(vb[6]), "r"(vb[7]), "r"(vb[8]),
+            "r"(vb[9]), "r"(vb[10]), "r"(vb[11]), "r"(vb[12]), "r"(vb[13]), "r"(vb[14]), "r"(vb[15]), "r"(vb[16]),
+            "r"(vb[17]), "r"(vb[18]), "r"(vb[19]), "r"(vb[20]), "r"(vb[21]), "r"(vb[22]), "r"(vb[23]), "r"(vb[24]),
+            "r"(vb[25]), "r"(vb[26]), "r"(vb[27]), "r"(vb[28]), "r"(vb[29]), "r"(vb[30]), "r"(vb[31]));
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) arrive_cluster(mapa(&sf_full[buf], 0));
+        if (++buf == NSF) { buf = 0; sph ^= 1; }
+        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------- epilogue --
+    constexpr int CW = OUT == OUT_F32 ? 32 : 64;
+    const int q = warp & 3, tid = threadIdx.x - 128, rl = q * 32 + lane;
+    uint32_t acc_ph = 0;
+    int chunk = 0;
+    const float tscale = __fmul_rn(*p.ta, *p.tb);
+    for (int64_t t = pair_id; t < ntiles; t += npairs) {
+      int64_t mb, nb;
+      tile_coords2(t, nm, nn, mb, nb);
+      const bool got = wait_c(acc_full, acc_ph, abort_flag, p.status);
+      if (epi_any(!got)) break;
+      acc_ph ^= 1;
+      tc_fence_after();
+      const int64_t row0 = mb * 256 + int64_t(rank) * 128, row = row0 + rl;
+      for (int c = 0; c < BN / CW; ++c) {
+        float v[CW];
+#pragma unroll
+        for (int i = 0; i < CW / 32; ++i)
+          tmem_ld32(tmem + ACC_COL + (uint32_t(q * 32) << 16) + c * CW + 32 * i, v + 32 * i);
+        if (c == BN / CW - 1) {                       // this CTA's accumulator half fully read
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) arrive_cluster(acc_empty_l);
+        }
+        const int64_t col0 = nb * BN + c * CW;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) v[j] = v[j] * tscale;
+        if (EPI == 1) {
+#pragma unroll
+          for (int hb = 0; hb < CW / 32; ++hb) {
+            float* u = v + 32 * hb;
+            const int64_t cb = col0 + 32 * hb;
+            if (p.mask && row < p.M && cb < p.N) {
+              const uint32_t mw = *reinterpret_cast<const uint32_t*>(p.mask + row * (p.N >> 3) + (cb >> 3));
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if ((mw >> j) & 1u) u[j] = 0.0f;
+            }
+#pragma unroll
+            for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                if (i & h) continue;
+                float a = u[i], b = u[i + h];
+                u[i] = a + b;
+                u[i + h] = a - b;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] *= 0.176776695296636881f;
+          }
+        }
+        uint32_t wds[32];
+        if (OUT == OUT_F32) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) wds[j] = __float_as_uint(v[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            wds[j] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+        }
+        uint8_t* stg = sStage + (chunk & 1) * STG_BYTES;
+        if (tid == 0) bulk_wait_read1();
+        epi_bar();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<uint4*>(stg + rl * 128 + ((j ^ (rl & 7)) << 4)) =
+              make_uint4(wds[4 * j], wds[4 * j + 1], wds[4 * j + 2], wds[4 * j + 3]);
+        fence_proxy_async();
+        epi_bar();
+        if (tid == 0 && row0 < p.M) {
+          tma_store_2d(&map_d, stg, int(col0), int(row0));
+          bulk_commit();
+        }
+        ++chunk;
+      }
+    }
+    if (tid == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();                                   // no arrivals or MMAs into the peer remain
+  if (warp == 2) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+}  // namespace pair
+
 // ------------------------------------------------------------ host side --
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -543,6 +942,37 @@ static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CU
   return cudaGetLastError();
 }
 
+// CTA-pair launch: one 2-CTA cluster per resident pair of SMs (as many as
+// the device co-schedules), grid-stride over the 256 x 256 tiles.
+template <int FMT, int OUT, int EPI>
+static cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
+                               const Params& p, cudaStream_t s) {
+  auto kern = pair::k_gemm_pair<FMT, OUT, EPI>;
+  static int max_clusters[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (max_clusters[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * unsigned(num_sms() / 2));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = pair::SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = num_sms() / 2;
+    }
+    max_clusters[dev] = n;
+  }
+  const int64_t tiles = ((p.M + 255) / 256) * ((p.N + BN - 1) / BN);
+  const int64_t pairs = tiles < max_clusters[dev] ? tiles : max_clusters[dev];
+  kern<<<unsigned(2 * pairs), THREADS, pair::SMEM_BYTES, s>>>(ma, mb, md, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace gemm
 }  // namespace fp4
 
@@ -572,9 +1002,14 @@ extern "C" int fp4_gemm(const fp4_qtensor* A, const fp4_qtensor* B, void* D, int
     size_t bytes = size_t(M) * size_t(N) * (out_dtype ? 2 : 4);
     return cudaMemsetAsync(D, 0, bytes, s) == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
   }
+  // Two-CTA (cta_group::2) kernel unless M fits one 128-row block, where the
+  // second CTA of every pair would have no rows.  FP4_GEMM_PAIR=0 in the
+  // environment selects the one-CTA kernel for every shape (read per call).
+  const char* pair_env = getenv("FP4_GEMM_PAIR");
+  const bool use_pair = M > gemm::BM && !(pair_env && pair_env[0] == '0');
   CUtensorMap ma, mb, md;
-  if (!gemm::make_map(&ma, A->codes, M, K, gemm::BM) || !gemm::make_map(&mb, B->codes, N, K, gemm::BN) ||
-      !gemm::make_map_d(&md, D, M, N, out_dtype))
+  if (!gemm::make_map(&ma, A->codes, M, K, gemm::BM) ||
+      !gemm::make_map(&mb, B->codes, N, K, use_pair ? 128 : gemm::BN) || !gemm::make_map_d(&md, D, M, N, out_dtype))
     return FP4_ERR_CUDA;
   gemm::Params p{};
   p.M = M; p.N = N; p.K = K;
@@ -584,12 +1019,15 @@ extern "C" int fp4_gemm(const fp4_qtensor* A, const fp4_qtensor* B, void* D, int
   p.D = D; p.mask = epi_mask; p.status = status_ptr();
   cudaError_t e;
   const bool nv = A->fmt == FP4_NVFP4, bf = out_dtype == 1, epi = epi_inverse_had == 32;
+#define FP4_GEMM_LAUNCH(F, O, E) \
+  (use_pair ? gemm::launch_pair<F, O, E>(ma, mb, md, p, s) : gemm::launch<F, O, E>(ma, mb, md, p, s))
   if (nv) {
-    if (bf) e = epi ? gemm::launch<1, 1, 1>(ma, mb, md, p, s) : gemm::launch<1, 1, 0>(ma, mb, md, p, s);
-    else e = epi ? gemm::launch<1, 0, 1>(ma, mb, md, p, s) : gemm::launch<1, 0, 0>(ma, mb, md, p, s);
+    if (bf) e = epi ? FP4_GEMM_LAUNCH(1, 1, 1) : FP4_GEMM_LAUNCH(1, 1, 0);
+    else e = epi ? FP4_GEMM_LAUNCH(1, 0, 1) : FP4_GEMM_LAUNCH(1, 0, 0);
   } else {
-    if (bf) e = epi ? gemm::launch<0, 1, 1>(ma, mb, md, p, s) : gemm::launch<0, 1, 0>(ma, mb, md, p, s);
-    else e = epi ? gemm::launch<0, 0, 1>(ma, mb, md, p, s) : gemm::launch<0, 0, 0>(ma, mb, md, p, s);
+    if (bf) e = epi ? FP4_GEMM_LAUNCH(0, 1, 1) : FP4_GEMM_LAUNCH(0, 1, 0);
+    else e = epi ? FP4_GEMM_LAUNCH(0, 0, 1) : FP4_GEMM_LAUNCH(0, 0, 0);
   }
+#undef FP4_GEMM_LAUNCH
   return e == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }

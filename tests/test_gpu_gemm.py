@@ -46,7 +46,10 @@ def check(y, y_ref, bound, rel_bf16=False):
 
 @pytest.mark.parametrize("fmt", [qn.NVFP4, qn.MXFP4])
 @pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 384, 512), (256, 264, 320), (64, 8, 64),
-                                   (1024, 1024, 1024)])
+                                   (1024, 1024, 1024),
+                                   # CTA-pair kernel (M > 128): second CTA's rows past M, B tile
+                                   # half past N, long K wrapping the 5-stage ring
+                                   (300, 136, 192), (384, 640, 1024), (512, 512, 4096), (136, 520, 64)])
 def test_gemm_parity(cuda_lib, fmt, M, N, K):
     A, B = operands(fmt, M, N, K, seed=M + N + K)
     y = cuda_lib.gemm(upload(cuda_lib, A), upload(cuda_lib, B))
