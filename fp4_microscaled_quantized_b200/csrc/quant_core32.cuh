@@ -444,10 +444,18 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
   uint32_t sm[LOAD == LD_ROW ? 16 : 4];
   if (LOAD == LD_ROW) sign_masks_bf16(sw, sm);
   else sign_masks_fp4(sw, sm);
-  for (int64_t base = int64_t(blockIdx.x) * blockDim.x + (threadIdx.x & ~31); base < tasks; base += stride) {
+  // Row and column task of t = base + lane, advanced by the grid stride
+  // without a division per task.
+  const int64_t base0 = int64_t(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
+  int64_t trow = (base0 + lane) / tpr, tct = (base0 + lane) % tpr;
+  const int64_t drow = stride / tpr, dct = stride % tpr;
+  for (int64_t base = base0; base < tasks; base += stride) {
     const int64_t t = base + lane;
     const bool active = t < tasks;
-    const int64_t orow = active ? t / tpr : 0, ocol = active ? (t % tpr) * 32 : 0;
+    const int64_t orow = active ? trow : 0, ocol = active ? tct * 32 : 0;
+    tct += dct;
+    trow += drow;
+    if (tct >= tpr) { tct -= tpr; ++trow; }
     float x[32];
     if (LOAD == LD_ROW) {
       const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + orow * p.cols + ocol);

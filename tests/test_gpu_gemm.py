@@ -58,6 +58,18 @@ def test_gemm_parity(cuda_lib, fmt, M, N, K):
 
 
 @pytest.mark.parametrize("fmt", [qn.NVFP4, qn.MXFP4])
+@pytest.mark.parametrize("M,N,K", [(300, 136, 192), (1024, 1024, 1024)])
+def test_gemm_one_cta_kernel(cuda_lib, monkeypatch, fmt, M, N, K):
+    """FP4_GEMM_PAIR=0 runs the one-CTA kernel on shapes that otherwise take
+    the CTA-pair kernel; both meet the bound."""
+    monkeypatch.setenv("FP4_GEMM_PAIR", "0")
+    A, B = operands(fmt, M, N, K, seed=M + N + K + 1)
+    y = cuda_lib.gemm(upload(cuda_lib, A), upload(cuda_lib, B))
+    y_ref, bound = gm.gemm_ref(A, B)
+    check(y, y_ref, bound)
+
+
+@pytest.mark.parametrize("fmt", [qn.NVFP4, qn.MXFP4])
 def test_gemm_lossless_exact(cuda_lib, fmt):
     """Grid values with power-of-two scales: every product and partial sum is
     exact in fp32, so the tensor-core result equals the exact product --
