@@ -94,8 +94,14 @@ def _sse(xg, codes, d):
     return fm.pairwise_sum((e * e).astype(F32))
 
 
-def _sr_index(rows, cols):
-    return np.arange(rows * cols, dtype=np.uint64).reshape(rows, cols)
+def _sr_index(rows, cols, row_ids=None):
+    """Linear element indices (the Philox counter of element SR): rows are
+    rows 0..rows-1 of the tensor, or the rows ``row_ids`` of a larger tensor
+    with the same number of columns."""
+    if row_ids is None:
+        return np.arange(rows * cols, dtype=np.uint64).reshape(rows, cols)
+    r = np.asarray(row_ids, dtype=np.uint64).reshape(rows, 1)
+    return r * np.uint64(cols) + np.arange(cols, dtype=np.uint64)[None, :]
 
 
 # ---------------------------------------------------------------- NVFP4 ----
@@ -144,7 +150,7 @@ def nvfp4_four_over_six(x, amax=None):
                    extra={"pick4": pick4})
 
 
-def nvfp4_sr(x, seed, tensor_tag, amax=None):
+def nvfp4_sr(x, seed, tensor_tag, amax=None, row_ids=None):
     """NVIDIA-style NVFP4 stochastic rounding (Quartet II page, "NVFP4 Format
     and Standard Stochastic Rounding", Steps 1-3): the 16/17 guard makes the
     normalised values stay within [-6, 6] so SR never clips."""
@@ -157,7 +163,7 @@ def nvfp4_sr(x, seed, tensor_tag, amax=None):
     s8 = fm.rtn_e4m3((gmax / F32(s32 * NV_SR_GROUP_DIV)).astype(F32))
     d = (fm.e4m3_value(s8).astype(F32) * s32).astype(F32)
     _, v, ok = _encode_rtn(xg, d)
-    u = philox.uniform(seed, _sr_index(rows, cols), philox.TAG_SR_ELEM, tensor_tag)
+    u = philox.uniform(seed, _sr_index(rows, cols, row_ids), philox.TAG_SR_ELEM, tensor_tag)
     codes = fm.sr_e2m1(v.reshape(rows, cols), u)
     codes = np.where(ok.repeat(16, axis=-1), codes, 0).astype(np.uint8)
     return QTensor(codes, s8, s32, NVFP4)
@@ -245,7 +251,7 @@ def ms_eden_tensor_scale(amax):
     return F32(np.ldexp(1.0, max(k, -126)))      # kept a normal fp32
 
 
-def ms_eden_pass2(p, S, amax, chunk, seed, tensor_tag):
+def ms_eden_pass2(p, S, amax, chunk, seed, tensor_tag, row_ids=None):
     """MS-EDEN second kernel: shift the pseudo-scales into the FP8 range by
     the power-of-two tensor scale, fold in the EDEN factor S of their
     rotation chunk and round to E4M3 stochastically (Algorithm 1 Step 4; post
@@ -255,8 +261,7 @@ def ms_eden_pass2(p, S, amax, chunk, seed, tensor_tag):
     inv32 = F32(F32(1.0) / s32)
     Sg = np.repeat(S, chunk // 16, axis=-1).astype(F32)
     t = ((Sg * p).astype(F32) * inv32).astype(F32)
-    u = philox.uniform(seed, np.arange(rows * ng, dtype=np.uint64).reshape(rows, ng),
-                       philox.TAG_SR_SCALE, tensor_tag)
+    u = philox.uniform(seed, _sr_index(rows, ng, row_ids), philox.TAG_SR_SCALE, tensor_tag)
     s8 = fm.sr_e4m3(t, u)
     return s8, s32
 
@@ -287,9 +292,12 @@ def ms_eden_algorithm1(y, chunk, seed, tensor_tag):
     return QTensor(codes.reshape(rows, cols), fm.sr_e4m3(t, u), s32, NVFP4)
 
 
-def nvfp4_ms_eden(y, chunk, seed, tensor_tag):
-    codes, p, S, amax = ms_eden_pass1(y, chunk)
-    s8, s32 = ms_eden_pass2(p, S, amax, chunk, seed, tensor_tag)
+def nvfp4_ms_eden(y, chunk, seed, tensor_tag, amax=None, row_ids=None):
+    """Both passes; ``amax`` (the global max |y| of the whole tensor) and
+    ``row_ids`` let a sample of the tensor's rows be quantised alone."""
+    codes, p, S, amax1 = ms_eden_pass1(y, chunk)
+    amax = amax1 if amax is None else F32(amax)
+    s8, s32 = ms_eden_pass2(p, S, amax, chunk, seed, tensor_tag, row_ids)
     return QTensor(codes, s8, s32, NVFP4, extra={"pseudo": p, "S": S, "amax": amax})
 
 
@@ -323,7 +331,7 @@ def mxfp4_rtn(x):
     return QTensor(codes.reshape(x.shape), (e + 127).astype(np.uint8), F32(1.0), MXFP4)
 
 
-def mxfp4_sr(x, seed, tensor_tag):
+def mxfp4_sr(x, seed, tensor_tag, row_ids=None):
     """Quartet backward quantizer G_q = SR(3/4 G_h) on MXFP4 (Quartet page,
     "Backward-Pass Quantization", the 3/4 rescaling factor).  READING: the
     exponent comes from the unscaled group max (OCP rule) and the values are
@@ -335,7 +343,7 @@ def mxfp4_sr(x, seed, tensor_tag):
     xg = _groups(x, 32)
     e = mx_exponent(_group_max(xg))
     v = ((xg * QUARTET_PRESCALE).astype(F32) * _pow2_f32(-e)[..., None]).astype(F32)
-    u = philox.uniform(seed, _sr_index(rows, cols), philox.TAG_SR_ELEM, tensor_tag)
+    u = philox.uniform(seed, _sr_index(rows, cols, row_ids), philox.TAG_SR_ELEM, tensor_tag)
     codes = fm.sr_e2m1(v.reshape(rows, cols), u)
     return QTensor(codes, (e + 127).astype(np.uint8), QUARTET_TENSOR_SCALE, MXFP4)
 
@@ -387,24 +395,27 @@ def supported(fmt, rnd, had_block):
     return True
 
 
-def quantize_transformed(y, fmt, rnd, seed=0, tensor_tag=0, chunk=None):
-    """Quantise an already transformed fp32 tensor (groups along cols)."""
+def quantize_transformed(y, fmt, rnd, seed=0, tensor_tag=0, chunk=None, amax=None, row_ids=None):
+    """Quantise an already transformed fp32 tensor (groups along cols).  For
+    a sample of a larger tensor's rows: ``amax`` is the whole tensor's max
+    |y| (NVFP4 tensor scale) and ``row_ids`` its row indices (Philox
+    counters); every other step is row-local."""
     if fmt == NVFP4:
         if rnd == RTN:
-            return nvfp4_rtn(y)
+            return nvfp4_rtn(y, amax)
         if rnd == FOUR_OVER_SIX:
-            return nvfp4_four_over_six(y)
+            return nvfp4_four_over_six(y, amax)
         if rnd == SR:
-            return nvfp4_sr(y, seed, tensor_tag)
+            return nvfp4_sr(y, seed, tensor_tag, amax, row_ids)
         if rnd == QUEST:
-            return nvfp4_quest(y)
+            return nvfp4_quest(y, amax)
         if rnd == MS_EDEN:
-            return nvfp4_ms_eden(y, chunk, seed, tensor_tag)
+            return nvfp4_ms_eden(y, chunk, seed, tensor_tag, amax, row_ids)
     else:
         if rnd == RTN:
             return mxfp4_rtn(y)
         if rnd == SR:
-            return mxfp4_sr(y, seed, tensor_tag)
+            return mxfp4_sr(y, seed, tensor_tag, row_ids)
         if rnd == QUEST:
             return mxfp4_quest(y)
     raise ValueError("unsupported format / rounding combination")
@@ -422,6 +433,37 @@ def quantize(x, fmt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0,
         a = np.ascontiguousarray(a.T)
     y = hd.block_transform(a, had_block, randomized, seed, sign_tag)
     return quantize_transformed(y, fmt, rnd, seed, tensor_tag, chunk=had_block)
+
+
+def transformed_abs_max(x, had_block=0, randomized=False, seed=0, sign_tag=0, transpose=False,
+                        rows_per_chunk=2048):
+    """max |y| of the whole transformed tensor y = block_transform(x or x^T),
+    computed a chunk of rows at a time (the rotation is row-local)."""
+    a = np.asarray(x).T if transpose else np.asarray(x)
+    m = F32(0.0)
+    for r0 in range(0, a.shape[0], rows_per_chunk):
+        y = hd.block_transform(np.ascontiguousarray(a[r0:r0 + rows_per_chunk], dtype=F32), had_block,
+                               randomized, seed, sign_tag)
+        m = max(m, abs_max(y))
+    return F32(m)
+
+
+def quantize_rows(x, rows, fmt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0,
+                  tensor_tag=0, transpose=False, amax=None):
+    """Rows ``rows`` of ``quantize(x, ...)`` (codes, scales, tensor scale),
+    from those rows of the (transposed) input alone: rotation, scales and
+    codes are row-local; NVFP4 also needs the whole transformed tensor's
+    max |y| (``amax``, computed here when not given) and the stochastic modes
+    index Philox by the rows' positions in the whole tensor."""
+    if not supported(fmt, rnd, had_block):
+        raise ValueError("unsupported format / rounding / Hadamard combination")
+    rows = np.asarray(rows, dtype=np.int64)
+    a = np.asarray(x).T if transpose else np.asarray(x)
+    sub = np.ascontiguousarray(a[rows], dtype=F32)
+    y = hd.block_transform(sub, had_block, randomized, seed, sign_tag)
+    if fmt == NVFP4 and amax is None:
+        amax = transformed_abs_max(x, had_block, randomized, seed, sign_tag, transpose)
+    return quantize_transformed(y, fmt, rnd, seed, tensor_tag, chunk=had_block, amax=amax, row_ids=rows)
 
 
 # ------------------------------------------------------- dequantisation ----
