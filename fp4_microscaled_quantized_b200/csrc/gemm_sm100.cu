@@ -500,6 +500,14 @@ constexpr int SFA_BYTES = 4 * 512;
 constexpr int SFB_BYTES = 8 * 512;                   // both 128-row blocks of the tile's B
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * STG_BYTES + 1024 + 256;
+// 16 warps: producer, MMA issuer, TMEM allocator, spare | 4 scale stagers |
+// 8 epilogue warps (two per TMEM lane quadrant, 128 columns each).  The
+// block launches with 128 registers a thread (65536); the first two
+// warpgroups give registers back so the epilogue can hold 128 accumulator
+// columns per thread: 128 x (56 + 80 + 184 + 184) = 64512 <= 65536.
+constexpr int PTHREADS = 512;
+constexpr int REG_CTRL = 56, REG_STAGE = 80, REG_EPI = 184;
+static_assert(128 * (REG_CTRL + REG_STAGE + 2 * REG_EPI) <= 65536, "register split of the CTA-pair kernel");
 static_assert(SMEM_BYTES <= 232448, "shared memory of the CTA-pair kernel");
 
 __device__ __forceinline__ uint32_t cta_rank() {
@@ -576,6 +584,12 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Named barrier of the four epilogue warps that cover one 128-column half.
+__device__ __forceinline__ void half_bar(int h) {
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
 template <int FMT>
 __device__ __forceinline__ void mma_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
                                          uint32_t sfb, uint32_t acc) {
@@ -605,7 +619,7 @@ __device__ __forceinline__ void tile_coords2(int64_t t, int64_t nm, int64_t nn, 
 }
 
 template <int FMT, int OUT, int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_d, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -641,7 +655,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       mbar_init(&sf_ld[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 8);
+    mbar_init(acc_empty, 16);
     for (int b = 0; b < NSF; ++b) { mbar_init(&sf_full[b], 8); mbar_init(&sf_empty[b], 1); }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -657,9 +671,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();                                   // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // warpgroup of this warp, warp-uniform for the compiler
+  const int wg = __shfl_sync(0xFFFFFFFFu, int(threadIdx.x) >> 7, 0);
   // the leader's barriers that both CTAs arrive on
   const uint32_t acc_empty_l = mapa(acc_empty, 0);
 
+  if (wg == 0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CTRL));
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------ TMA producer --
     int s = 0;
@@ -733,7 +751,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const unsigned long long t0 = clock64();
       while (!try_c(drain, 0) && clock64() - t0 < WAIT_LIMIT) {}
     }
-  } else if (warp >= 8) {
+  }
+  } else if (wg == 1) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_STAGE));
     // ------------------------------------------- scale factors -> TMEM --
     const int q = warp & 3;
     int s = 0, buf = 0;
@@ -780,87 +800,98 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (++s == STAGES) { s = 0; ph ^= 1; }
       }
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_EPI));
     // ---------------------------------------------------------- epilogue --
+    // warp 8 + 4h + q holds TMEM lane quadrant q (rows 32q..32q+31 of this
+    // CTA's half) and columns 128h .. 128h+127: all of them are read into
+    // registers and the accumulator is released (on the leader's
+    // acc_empty) before any store, so the next tile's MMAs overlap the
+    // stores; then the four warps of half h store 32-column (fp32) or
+    // 64-column (bf16) chunks through the half's 128-byte-swizzled staging
+    // buffer with TMA stores.
     constexpr int CW = OUT == OUT_F32 ? 32 : 64;
-    const int q = warp & 3, tid = threadIdx.x - 128, rl = q * 32 + lane;
+    const int q = warp & 3, h = (warp - 8) >> 2, rl = q * 32 + lane;
+    const bool storer = q == 0 && lane == 0;        // one thread per half issues its stores
+    uint8_t* stg = sStage + h * STG_BYTES;
     uint32_t acc_ph = 0;
-    int chunk = 0;
     const float tscale = __fmul_rn(*p.ta, *p.tb);
     for (int64_t t = pair_id; t < ntiles; t += npairs) {
       int64_t mb, nb;
       tile_coords2(t, nm, nn, mb, nb);
       const bool got = wait_c(acc_full, acc_ph, abort_flag, p.status);
-      if (epi_any(!got)) break;
+      uint32_t bad;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+          "bar.red.or.pred q, 3, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(bad)
+          : "r"(uint32_t(!got))
+          : "memory");
+      if (bad) break;                                // uniform across the 8 epilogue warps
       acc_ph ^= 1;
       tc_fence_after();
+      float v[128];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_ld32(tmem + ACC_COL + (uint32_t(q * 32) << 16) + 128 * h + 32 * i, v + 32 * i);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) arrive_cluster(acc_empty_l);
       const int64_t row0 = mb * 256 + int64_t(rank) * 128, row = row0 + rl;
-      for (int c = 0; c < BN / CW; ++c) {
-        float v[CW];
 #pragma unroll
-        for (int i = 0; i < CW / 32; ++i)
-          tmem_ld32(tmem + ACC_COL + (uint32_t(q * 32) << 16) + c * CW + 32 * i, v + 32 * i);
-        if (c == BN / CW - 1) {                       // this CTA's accumulator half fully read
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) arrive_cluster(acc_empty_l);
-        }
-        const int64_t col0 = nb * BN + c * CW;
+      for (int j = 0; j < 128; ++j) v[j] = v[j] * tscale;
+      if (EPI == 1) {
 #pragma unroll
-        for (int j = 0; j < CW; ++j) v[j] = v[j] * tscale;
-        if (EPI == 1) {
+        for (int hb = 0; hb < 4; ++hb) {
+          float* u = v + 32 * hb;
+          const int64_t cb = nb * BN + 128 * h + 32 * hb;
+          if (p.mask && row < p.M && cb < p.N) {
+            const uint32_t mw = *reinterpret_cast<const uint32_t*>(p.mask + row * (p.N >> 3) + (cb >> 3));
 #pragma unroll
-          for (int hb = 0; hb < CW / 32; ++hb) {
-            float* u = v + 32 * hb;
-            const int64_t cb = col0 + 32 * hb;
-            if (p.mask && row < p.M && cb < p.N) {
-              const uint32_t mw = *reinterpret_cast<const uint32_t*>(p.mask + row * (p.N >> 3) + (cb >> 3));
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if ((mw >> j) & 1u) u[j] = 0.0f;
-            }
-#pragma unroll
-            for (int h = 1; h < 32; h <<= 1) {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                if (i & h) continue;
-                float a = u[i], b = u[i + h];
-                u[i] = a + b;
-                u[i + h] = a - b;
-              }
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] *= 0.176776695296636881f;
+            for (int j = 0; j < 32; ++j)
+              if ((mw >> j) & 1u) u[j] = 0.0f;
           }
+#pragma unroll
+          for (int hh = 1; hh < 32; hh <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (i & hh) continue;
+              float a = u[i], b = u[i + hh];
+              u[i] = a + b;
+              u[i + hh] = a - b;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) u[j] *= 0.176776695296636881f;
         }
+      }
+#pragma unroll
+      for (int c = 0; c < 128 / CW; ++c) {
         uint32_t wds[32];
         if (OUT == OUT_F32) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) wds[j] = __float_as_uint(v[j]);
+          for (int j = 0; j < 32; ++j) wds[j] = __float_as_uint(v[CW * c + j]);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(v[CW * c + 2 * j], v[CW * c + 2 * j + 1]);
             wds[j] = *reinterpret_cast<uint32_t*>(&h2);
           }
         }
-        uint8_t* stg = sStage + (chunk & 1) * STG_BYTES;
-        if (tid == 0) bulk_wait_read1();
-        epi_bar();
+        if (storer) bulk_wait_read0();               // the previous store has read the buffer
+        half_bar(h);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           *reinterpret_cast<uint4*>(stg + rl * 128 + ((j ^ (rl & 7)) << 4)) =
               make_uint4(wds[4 * j], wds[4 * j + 1], wds[4 * j + 2], wds[4 * j + 3]);
         fence_proxy_async();
-        epi_bar();
-        if (tid == 0 && row0 < p.M) {
-          tma_store_2d(&map_d, stg, int(col0), int(row0));
+        half_bar(h);
+        if (storer && row0 < p.M) {
+          tma_store_2d(&map_d, stg, int(nb * BN + 128 * h + CW * c), int(row0));
           bulk_commit();
         }
-        ++chunk;
       }
     }
-    if (tid == 0) bulk_wait_all();
+    if (storer) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -957,7 +988,7 @@ static cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, con
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * unsigned(num_sms() / 2));
-    cfg.blockDim = dim3(THREADS);
+    cfg.blockDim = dim3(pair::PTHREADS);
     cfg.dynamicSmemBytes = pair::SMEM_BYTES;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
@@ -968,7 +999,7 @@ static cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, con
   }
   const int64_t tiles = ((p.M + 255) / 256) * ((p.N + BN - 1) / BN);
   const int64_t pairs = tiles < max_clusters[dev] ? tiles : max_clusters[dev];
-  kern<<<unsigned(2 * pairs), THREADS, pair::SMEM_BYTES, s>>>(ma, mb, md, p);
+  kern<<<unsigned(2 * pairs), pair::PTHREADS, pair::SMEM_BYTES, s>>>(ma, mb, md, p);
   count_launch();
   return cudaGetLastError();
 }
