@@ -261,7 +261,8 @@ class Step:
 def run_e2e(api, M, steps, device, host):
     """Same metric through the public linear-layer API with host buffers:
     every step copies X, W, dY of every layer host->device (pinned), runs
-    fp4_linear_fwd + fp4_linear_bwd and reads dW back device->host."""
+    fp4_linear_fwd + fp4_linear_bwd and reads dW back device->host, the
+    copies overlapped with the other layers' compute."""
     r = api.recipe(api.RECIPE_QUARTET2)
     devbuf = []
     for li, (name, K, N) in enumerate(LAYERS):
@@ -278,21 +279,47 @@ def run_e2e(api, M, steps, device, host):
     h2d = sum(v.numel() * v.element_size() for h in host for v in h.values())
     d2h = sum(b["dW"].numel() * 4 for b in devbuf)
 
-    def step(seed):
-        for h, b in zip(host, devbuf):
-            for k in ("X", "W", "dY"):
-                b[k].copy_(h[k], non_blocking=True)
+    # Host->device and device->host copies run on their own streams: every
+    # layer's inputs stream in while earlier layers compute, and each dW
+    # streams out while later layers compute.  Each layer has its own device
+    # buffers; the next step's copy into them waits for this step's use.
+    comp = torch.cuda.current_stream()
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(devbuf)
+    ev_in = [torch.cuda.Event() for _ in range(n)]
+    ev_done = [torch.cuda.Event() for _ in range(n)]
+    ev_d2h = [torch.cuda.Event() for _ in range(n)]
+    ev_out = torch.cuda.Event()
+
+    def step(seed, first):
+        for i, (h, b) in enumerate(zip(host, devbuf)):
+            with torch.cuda.stream(cin):
+                if not first:
+                    cin.wait_event(ev_done[i])
+                for k in ("X", "W", "dY"):
+                    b[k].copy_(h[k], non_blocking=True)
+                ev_in[i].record(cin)
+        for i, b in enumerate(devbuf):
+            comp.wait_event(ev_in[i])
+            if not first:
+                comp.wait_event(ev_d2h[i])         # last step's dW has left this buffer
             api.linear_fwd(b["X"], b["W"], r, 0, ctx=b["ctx"], Y=b["Y"], ws=b["wsf"])
             api.linear_bwd(b["dY"], b["ctx"], seed, dX=b["dX"], dW=b["dW"], ws=b["wsb"])
-            b["dW_host"].copy_(b["dW"], non_blocking=True)
+            ev_done[i].record(comp)
+            with torch.cuda.stream(cout):
+                cout.wait_event(ev_done[i])
+                b["dW_host"].copy_(b["dW"], non_blocking=True)
+                ev_d2h[i].record(cout)
+        ev_out.record(cout)
 
-    step(0)
+    step(0, True)
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
+    s.record(comp)
     for k in range(steps):
-        step(100 + k)
-    e.record()
+        step(100 + k, k == 0)
+    comp.wait_event(ev_out)                      # the last dW is on the host
+    e.record(comp)
     torch.cuda.synchronize()
     ms = s.elapsed_time(e) / steps
     flops = sum(6.0 * M * N * K for _, K, N in LAYERS)
