@@ -54,6 +54,14 @@ def parse():
     ap.add_argument("--tokens", type=int, default=M_TOKENS)
     ap.add_argument("--layers", default="qkv,o,gate_up,down",
                     help="subset of the layer set (profiling small cases)")
+    ap.add_argument("--quant-sweep", action="store_true",
+                    help="quantiser-only sweep (formats x rounding modes x Hadamard blocks x sizes) "
+                         "instead of the layer-set step")
+    ap.add_argument("--sweep-log2", default="20,22,24,26,28,30",
+                    help="log2 element counts of the sweep tensors (rows of 4096)")
+    ap.add_argument("--sweep-cases", default="all",
+                    help="comma list of sweep case names (e.g. nvfp4-fos-h0,nvfp4-eden-h128) or 'all'")
+    ap.add_argument("--sweep-reps", type=int, default=10)
     args = ap.parse_args()
     global LAYERS
     keep = args.layers.split(",")
@@ -329,6 +337,105 @@ def run_e2e(api, M, steps, device, host):
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
 
 
+# ------------------------------------------------------ quantiser sweep --
+SWEEP_COLS = 4096
+RND_NAMES = {0: "rtn", 1: "quest", 2: "fos", 3: "sr", 4: "eden"}
+
+
+def sweep_cases(api):
+    """(name, fmt, rounding, had_block, randomized) of every combination the C ABI
+    accepts: MXFP4 (RTN, QuEST, SR) and NVFP4 (RTN, QuEST, 4/6, SR) with Hadamard
+    none/16/32/128, NVFP4 MS-EDEN with 16/32/128.  The stochastic modes use the
+    randomized transform (backward pass), the others the deterministic one."""
+    out = []
+    for fmt, fname, rnds in ((api.MXFP4, "mxfp4", (api.RTN, api.QUEST, api.SR)),
+                             (api.NVFP4, "nvfp4", (api.RTN, api.QUEST, api.FOUR_OVER_SIX, api.SR,
+                                                   api.MS_EDEN))):
+        for rnd in rnds:
+            for had in (0, 16, 32, 128):
+                if rnd == api.MS_EDEN and had == 0:
+                    continue
+                rand = rnd in (api.SR, api.MS_EDEN) and had > 0
+                out.append(("%s-%s-h%d" % (fname, RND_NAMES[rnd], had), fmt, rnd, had, rand))
+    return out
+
+
+def sweep_bytes_per_elem(api, fmt, rnd, had):
+    """Algorithmic HBM bytes per element of one quantise call: bf16 read 2 B,
+    codes 0.5, one scale copy 1/g; NVFP4 global-scale modes read the input
+    twice (amax pass); QuEST writes a 1-bit mask; MS-EDEN writes and re-reads
+    bf16 pseudo-scales (2 x 2/16) and fp32 EDEN factors (2 x 4/had)."""
+    g = api.GROUP[fmt]
+    b = 2.0 + 0.5 + 1.0 / g
+    if fmt == api.NVFP4 and rnd != api.MS_EDEN:
+        b += 2.0
+    if rnd == api.QUEST:
+        b += 1.0 / 8
+    if rnd == api.MS_EDEN:
+        b += 2 * 2.0 / 16 + 2 * 4.0 / had
+    return b
+
+
+def quant_sweep(args):
+    """Config-5 sweep: every quantiser combination on N(0,1) + 0.1% x50
+    outlier tensors of 2^n bf16 elements (rows of 4096), row-wise.  Each call
+    is timed alone with CUDA events on the launching stream, the L2 flushed
+    (a 256 MiB write) before every repetition; one JSON line per case."""
+    from fp4_microscaled_quantized_b200 import api
+    api.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, src = load_peaks()
+    logs = [int(s) for s in args.sweep_log2.split(",")]
+    cases = sweep_cases(api)
+    if args.sweep_cases != "all":
+        keep = set(args.sweep_cases.split(","))
+        cases = [c for c in cases if c[0] in keep]
+    rows_max = (1 << max(logs)) // SWEEP_COLS
+    # One seeded tensor of up to 2^28 elements; smaller sizes are its leading
+    # rows, larger ones repeat it (host generation of 2^30 draws takes minutes).
+    rows_gen = min(rows_max, (1 << 28) // SWEEP_COLS)
+    bits = syn.outlier_elements((rows_gen, SWEEP_COLS), seed=7)
+    x_gen = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    del bits
+    x_all = x_gen.repeat((rows_max + rows_gen - 1) // rows_gen, 1)[:rows_max] if rows_max > rows_gen else x_gen
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for lg in logs:
+        rows = (1 << lg) // SWEEP_COLS
+        x = x_all[:rows]
+        for name, fmt, rnd, had, rand in cases:
+            out = api.alloc_qtensor(rows, SWEEP_COLS, fmt, linear=False, mask=(rnd == api.QUEST),
+                                    device=dev)
+            ws = api.alloc_workspace(api.workspace_size(rows, SWEEP_COLS, fmt, rnd, had), dev)
+            call = lambda s: api.quantize(x, fmt, rnd, had, rand, s, 0, 1, out=out, ws=ws)  # noqa: E731
+            lc0 = api.launch_count()
+            for w in range(3):
+                call(w)
+            launches = (api.launch_count() - lc0) // 3
+            ts = []
+            for k in range(args.sweep_reps):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                call(100 + k)
+                b.record(stream)
+                b.synchronize()
+                ts.append(a.elapsed_time(b))
+            ms = float(np.median(ts))
+            n = rows * SWEEP_COLS
+            gbs = n * sweep_bytes_per_elem(api, fmt, rnd, had) / (ms * 1e-3) / 1e9
+            print(json.dumps({"case": name, "log2_elems": lg, "elems": n, "us": round(ms * 1e3, 2),
+                              "gb_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 3),
+                              "bytes_per_elem": sweep_bytes_per_elem(api, fmt, rnd, had),
+                              "launches": int(launches), "peak": "%s copy %.0f GB/s" % (src, peaks["hbm_gbs"])}),
+                  flush=True)
+            del out, ws
+    if api.get_last_error() != 0:
+        raise SystemExit("device status %d after the sweep" % api.get_last_error())
+
+
 # --------------------------------------------------------- CPU oracle --
 def oracle_sample(n_rows, n_out, seed=0):
     """The oracle's fwd+bwd on a bounded sample of the same workload: the
@@ -397,6 +504,10 @@ def main():
     if args.impl == "reference":
         reference_arm(args, world, rank)
         return
+    if args.quant_sweep:
+        if rank == 0:
+            quant_sweep(args)
+        return
     from fp4_microscaled_quantized_b200 import api
     api.load()
     dev = torch.device("cuda", local)
@@ -412,7 +523,7 @@ def main():
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
-    lc0 = api.load().fp4_launch_count()
+    lc0 = api.launch_count()
     step.records = []
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
@@ -420,7 +531,7 @@ def main():
         step.run(k)
     end.record()
     torch.cuda.synchronize()
-    lc1 = api.load().fp4_launch_count()
+    lc1 = api.launch_count()
     barrier(world)
     torch.cuda.synchronize()
     clk = clocks.stop()

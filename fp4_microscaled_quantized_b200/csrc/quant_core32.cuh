@@ -11,19 +11,40 @@
 
 namespace fp4 {
 
+// Hardware E2M1 conversion (round to nearest even, saturating at +-6) of two
+// values into bits 0-7 of the result (`lo` in bits 0-3, bits 8-31 zero).
+// The conversion writes a one-byte register.  Bytes cross the asm boundary
+// only inside a full 32-bit register whose other bytes are zero: one-byte
+// operands taken from wider registers (a four-way split of a word, or the
+// upper half of one) were read from the wrong byte in some kernels.
+__device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t.reg .b16 h;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+      "mov.b16 h, {t, 0};\n\t"
+      "cvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+// f16x2 grid values of the two codes in bits 0-7 of `b` (bits 8-31 zero;
+// bits 0-3 -> low half).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t b) {
+  uint32_t h;
+  asm("{\n\t.reg .b8 t, z;\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "mov.b16 {t, z}, lo;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(h) : "r"(b));
+  return h;
+}
+
 // E2M1 RTN of 8 values into one word (element j in bits 4j..4j+3) with the
-// hardware conversion (round to nearest even, saturating at +-6); negative
-// zeros are then cleared so a value rounding to 0 encodes as +0.
+// hardware conversion; negative zeros are then cleared so a value rounding
+// to 0 encodes as +0.
 __device__ __forceinline__ uint32_t enc8_hw(const float* v) {
-  uint32_t w;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(w)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  const uint32_t w = e2m1x2_rn(v[0], v[1]) | (e2m1x2_rn(v[2], v[3]) << 8) | (e2m1x2_rn(v[4], v[5]) << 16) |
+                     (e2m1x2_rn(v[6], v[7]) << 24);
   const uint32_t nz = ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;  // bit 3 set iff mag != 0
   return w & (nz | 0x77777777u);
 }
@@ -92,35 +113,30 @@ __device__ __forceinline__ void enc16(const float* x, float inv, bool ok, uint32
 }
 
 // Signed grid values of the 8 codes of a word (element j from bits 4j..4j+3):
-// the packed E2M1 -> f16x2 conversion, then f16 -> f32, both exact.  Code 8
-// gives -0.
+// the packed E2M1 -> f16x2 conversion of each byte, then f16 -> f32, both
+// exact.  Code 8 gives -0.
 __device__ __forceinline__ void dec8(uint32_t w, float* q) {
-  uint32_t h[4];
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(w));
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[k]));
+    const uint32_t h = e2m1x2_to_f16x2((w >> (8 * k)) & 0xFFu);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
     q[2 * k] = f.x;
     q[2 * k + 1] = f.y;
   }
 }
 
 // fp32 squared error of 16 elements against codes * d, pairwise tree:
-// e = x - fp32(q d), s = fp32(e e).
+// e = x - fp32(q d), s = fp32(e e).  The subtraction is a scalar IEEE
+// operation: a packed subtraction of a packed product can be fused into one
+// multiply-add by the code generator, which changes the rounding.
 __device__ __forceinline__ float sse16(const float* x, const uint32_t* w, float d) {
   float q[16], s[16];
   dec8(w[0], q);
   dec8(w[1], q + 8);
 #pragma unroll
   for (int j = 0; j < 16; j += 2) {
-    const float2 e = sub2(ld2(x, j), __fmul2_rn(ld2(q, j), splat2(d)));
+    const float2 qd = __fmul2_rn(ld2(q, j), splat2(d));
+    const float2 e = make_float2(__fsub_rn(x[j], qd.x), __fsub_rn(x[j + 1], qd.y));
     st2(s, j, __fmul2_rn(e, e));
   }
   return tree16p(s);
@@ -593,9 +609,12 @@ static __global__ void k_selftest_e2m1(unsigned long long* mismatches) {
   if (blockIdx.x == 0) {
     for (uint32_t c = threadIdx.x; c < 256u; c += blockDim.x) {
       float q[8];
-      dec8(c | (c << 8) | (c << 16) | (c << 24), q);
+      // four different bytes per word, so a byte decoded from the wrong
+      // position is seen
+      const uint32_t by[4] = {c, (c * 7u + 0x35u) & 0xFFu, c ^ 0xA6u, (c * 13u + 0x5Bu) & 0xFFu};
+      dec8(by[0] | (by[1] << 8) | (by[2] << 16) | (by[3] << 24), q);
       for (int j = 0; j < 8; ++j)
-        bad += (fbits(q[j]) != fbits(e2m1_value((c >> (4 * (j & 1))) & 15u))) ? 1ull : 0ull;
+        bad += (fbits(q[j]) != fbits(e2m1_value((by[j >> 1] >> (4 * (j & 1))) & 15u))) ? 1ull : 0ull;
     }
   }
   if (bad) atomicAdd(mismatches, bad);

@@ -10,13 +10,32 @@ cudaError_t launch_quant(int fmt, int rnd, int had, const QParams& p, cudaStream
 
 int num_sms();
 
+// Resident 256-thread blocks per SM of one row kernel (its registers and
+// shared memory decide), cached per instantiation and device: grid-stride
+// kernels launch exactly one full wave, so no block waits for a second wave
+// and then runs alone at the end.
+template <bool WIDE, int LOAD, int FMT, int RND, int HAD>
+int resident_blocks() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaError_t e = WIDE ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row32<LOAD, FMT, RND, HAD>, 256, 0)
+                         : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row<LOAD, FMT, RND, HAD>, 256, 0);
+    cached[dev] = (e == cudaSuccess && n >= 1) ? n : 1;
+  }
+  return cached[dev];
+}
+
 template <int LOAD, int FMT, int RND, int HAD>
 cudaError_t launch_one(const QParams& p, cudaStream_t s) {
   const bool wide = (p.cols % 32) == 0;   // 32 elements per lane
   if ((LOAD == LD_ROW || LOAD == LD_ROW_FP4) && wide) {
     int64_t tasks = p.rows * (p.cols >> 5);
     int64_t blocks = (tasks + 255) / 256;
-    int64_t cap = int64_t(num_sms()) * 4;
+    int64_t cap = int64_t(num_sms()) * resident_blocks<true, LOAD, FMT, RND, HAD>();
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     k_quant_row32<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
@@ -29,7 +48,7 @@ cudaError_t launch_one(const QParams& p, cudaStream_t s) {
   } else if (LOAD == LD_ROW || LOAD == LD_ROW_FP4) {
     int64_t tasks = p.rows * (p.cols >> 3);
     int64_t blocks = (tasks + 255) / 256;
-    int64_t cap = int64_t(num_sms()) * 8;
+    int64_t cap = int64_t(num_sms()) * resident_blocks<false, LOAD, FMT, RND, HAD>();
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     k_quant_row<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
