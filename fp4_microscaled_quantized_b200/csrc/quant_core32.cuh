@@ -486,11 +486,11 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
     } else {
       uint4 cw = make_uint4(0, 0, 0, 0);
       uint32_t s0 = 0, s1 = 0;
-      const int gin = p.in_fmt == FMT_NV ? 16 : 32;
+      const int gsh = p.in_fmt == FMT_NV ? 4 : 5;   // log2 of the input group size
       if (active) {
         cw = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) + orow * (p.cols >> 1) + (ocol >> 1)));
-        s0 = p.in_scales[orow * (p.cols / gin) + ocol / gin];
-        s1 = p.in_scales[orow * (p.cols / gin) + (ocol + 16) / gin];
+        s0 = p.in_scales[orow * (p.cols >> gsh) + (ocol >> gsh)];
+        s1 = p.in_scales[orow * (p.cols >> gsh) + ((ocol + 16) >> gsh)];
       }
       const float sa = fp4_in_scale(s0, p.in_fmt), sbv = fp4_in_scale(s1, p.in_fmt);
       const uint32_t cws[4] = {cw.x ^ sm[0], cw.y ^ sm[1], cw.z ^ sm[2], cw.w ^ sm[3]};
@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
     } else {
       const uint8_t* xc = static_cast<const uint8_t*>(p.x);
       const float in_ts = *p.in_ts;
-      const int gin = p.in_fmt == FMT_NV ? 16 : 32;
+      const int gsh = p.in_fmt == FMT_NV ? 4 : 5;   // log2 of the input group size
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int64_t r = r0 + rl + q;
@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
         uint32_t sa = 0;
         if (r < R && cc < C) {
           cw = __ldg(reinterpret_cast<const uint2*>(xc + r * (C >> 1) + (cc >> 1)));
-          sa = p.in_scales[r * (C / gin) + cc / gin];
+          sa = p.in_scales[r * (C >> gsh) + (cc >> gsh)];
         }
         const uint32_t m = (q ? sgn_b : sgn_a) * 0x88888888u;
         const float s_a = fp4_in_scale(sa, p.in_fmt);

@@ -379,8 +379,8 @@ __global__ void __launch_bounds__(256) k_quant_row(QParams p) {
       uint32_t cw = 0, sc = 0;
       if (active) {
         cw = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(p.x) + orow * (p.cols >> 1) + (ocol >> 1)));
-        int gin = p.in_fmt == FMT_NV ? 16 : 32;
-        sc = p.in_scales[orow * (p.cols / gin) + ocol / gin];
+        const int gsh = p.in_fmt == FMT_NV ? 4 : 5;   // log2 of the input group size
+        sc = p.in_scales[orow * (p.cols >> gsh) + (ocol >> gsh)];
       }
       float s = fp4_in_scale(sc, p.in_fmt);
 #pragma unroll
@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(256) k_quant_trans(QParams p) {
     } else {
       const uint8_t* xc = static_cast<const uint8_t*>(p.x);
       const float in_ts = *p.in_ts;
-      const int gin = p.in_fmt == FMT_NV ? 16 : 32;
+      const int gsh = p.in_fmt == FMT_NV ? 4 : 5;   // log2 of the input group size
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         int64_t r = r0 + rl + q;
@@ -433,8 +433,8 @@ __global__ void __launch_bounds__(256) k_quant_trans(QParams p) {
         uint32_t sa = 0, sb = 0;
         if (r < R && cc < C) {
           cw = __ldg(reinterpret_cast<const uint2*>(xc + r * (C >> 1) + (cc >> 1)));
-          sa = p.in_scales[r * (C / gin) + cc / gin];
-          sb = p.in_scales[r * (C / gin) + (cc + 8) / gin];
+          sa = p.in_scales[r * (C >> gsh) + (cc >> gsh)];
+          sb = p.in_scales[r * (C >> gsh) + ((cc + 8) >> gsh)];
         }
         float s_a = fp4_in_scale(sa, p.in_fmt), s_b = fp4_in_scale(sb, p.in_fmt);
         float* dst = q ? vb : va;
@@ -476,25 +476,34 @@ __global__ void __launch_bounds__(256) k_eden_pass2(QParams p) {
   const int64_t ng = p.cols >> 4, total = p.rows * ng;
   const float s32 = eden_tensor_scale(*p.amax_bits);
   const float inv32 = __frcp_rn(s32);
+  const int64_t ns = p.cols / HAD;                 // EDEN factors per row
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.ts = s32;
   if ((ng & 3) == 0) {
-    // four groups k0..k0+3 of one row per thread: one Philox block, 4-byte stores
-    for (int64_t q = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; q < (total >> 2);
-         q += int64_t(gridDim.x) * blockDim.x) {
-      const int64_t gi0 = q << 2, r = gi0 / ng, k0 = gi0 % ng;
+    // four groups k0..k0+3 of one row per thread: one Philox block, 4-byte
+    // stores; the (row, group) of each task advances by the grid stride
+    const int64_t nq = ng >> 2, stride = int64_t(gridDim.x) * blockDim.x;
+    const int64_t q0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    int64_t r = q0 / nq, kq = q0 % nq;
+    const int64_t dr = stride / nq, dk = stride % nq;
+    for (int64_t q = q0; q < (total >> 2); q += stride) {
+      const int64_t k0 = kq << 2, gi0 = q << 2;
       const uint2 ps = *reinterpret_cast<const uint2*>(p.pseudo + gi0);
-      const uint32_t pw[4] = {ps.x & 0xFFFFu, ps.x >> 16, ps.y & 0xFFFFu, ps.y >> 16};
+      const uint32_t pw[4] = {ps.x << 16, ps.x & 0xFFFF0000u, ps.y << 16, ps.y & 0xFFFF0000u};
       const u32x4 rb = philox_block(p.seed, uint64_t(q), TAG_SR_SCALE, p.tensor_tag);
       const uint32_t rw[4] = {rb.x, rb.y, rb.z, rb.w};
+      const float* Srow = p.eden_S + r * ns + (k0 * 16) / HAD;
       uint32_t word = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float S = p.eden_S[r * (p.cols / HAD) + ((k0 + j) * 16) / HAD];
-        const float t = __fmul_rn(__fmul_rn(S, bitsf(pw[j] << 16)), inv32);
-        word |= e4m3_sr(t, u24(rw[j])) << (8 * j);
+        const float S = Srow[(j * 16) / HAD];        // one factor per HAD / 16 groups
+        const float t = __fmul_rn(__fmul_rn(S, bitsf(pw[j])), inv32);
+        word |= e4m3_sr_bits(t, rw[j] >> 8) << (8 * j);
       }
       if (p.scales) *reinterpret_cast<uint32_t*>(p.scales + gi0) = word;
       if (p.swz) *reinterpret_cast<uint32_t*>(p.swz + swz_offset(r, k0, p.nkb)) = word;
+      kq += dk;
+      r += dr;
+      if (kq >= nq) { kq -= nq; ++r; }
     }
     return;
   }
@@ -502,9 +511,9 @@ __global__ void __launch_bounds__(256) k_eden_pass2(QParams p) {
        gi += int64_t(gridDim.x) * blockDim.x) {
     int64_t r = gi / ng, k = gi % ng;
     float pq = bitsf(uint32_t(p.pseudo[gi]) << 16);
-    float S = p.eden_S[r * (p.cols / HAD) + (k * 16) / HAD];
+    float S = p.eden_S[r * ns + (k * 16) / HAD];
     float t = __fmul_rn(__fmul_rn(S, pq), inv32);
-    uint32_t s8 = e4m3_sr(t, u24(philox_word(p.seed, uint64_t(gi), TAG_SR_SCALE, p.tensor_tag)));
+    uint32_t s8 = e4m3_sr_bits(t, philox_word(p.seed, uint64_t(gi), TAG_SR_SCALE, p.tensor_tag) >> 8);
     if (p.scales) p.scales[gi] = uint8_t(s8);
     if (p.swz) p.swz[swz_offset(r, k, p.nkb)] = uint8_t(s8);
   }
