@@ -275,6 +275,14 @@ int fp4_selftest_e2m1(unsigned long long* mismatches, fp4_stream_t stream) {
   return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
+int fp4_selftest_arith(unsigned long long* mismatches, fp4_stream_t stream) {
+  if (!mismatches) return FP4_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  k_selftest_arith<<<unsigned(num_sms() * 8), 256, 0, s>>>(mismatches);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
 const char* fp4_status_string(int st) {
   switch (st) {
     case FP4_OK: return "ok";

@@ -39,15 +39,24 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t b) {
   return h;
 }
 
-// E2M1 RTN of 8 values into one word (element j in bits 4j..4j+3) with the
-// hardware conversion; negative zeros are then cleared so a value rounding
-// to 0 encodes as +0.
-__device__ __forceinline__ uint32_t enc8_hw(const float* v) {
-  const uint32_t w = e2m1x2_rn(v[0], v[1]) | (e2m1x2_rn(v[2], v[3]) << 8) | (e2m1x2_rn(v[4], v[5]) << 16) |
-                     (e2m1x2_rn(v[6], v[7]) << 24);
+// Clear negative-zero codes (a value rounding to 0 is stored as +0).
+__device__ __forceinline__ uint32_t clear_neg_zero(uint32_t w) {
   const uint32_t nz = ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;  // bit 3 set iff mag != 0
   return w & (nz | 0x77777777u);
 }
+
+// E2M1 RTN of 8 values into one word (element j in bits 4j..4j+3) with the
+// hardware conversion, negative zeros kept (they decode to -0, which changes
+// no error or inner product); the four bytes are joined by byte permutes.
+__device__ __forceinline__ uint32_t enc8_raw(const float* v) {
+  const uint32_t lo = __byte_perm(e2m1x2_rn(v[0], v[1]), e2m1x2_rn(v[2], v[3]), 0x0040u);
+  const uint32_t hi = __byte_perm(e2m1x2_rn(v[4], v[5]), e2m1x2_rn(v[6], v[7]), 0x0040u);
+  return __byte_perm(lo, hi, 0x5410u);
+}
+
+// The stored form: negative zeros cleared so a value rounding to 0 encodes
+// as +0.
+__device__ __forceinline__ uint32_t enc8_hw(const float* v) { return clear_neg_zero(enc8_raw(v)); }
 
 // Software reference of the same word (the per-element encoder).
 __device__ __forceinline__ uint32_t enc8_sw(const float* v) {
@@ -103,13 +112,19 @@ __device__ __forceinline__ uint32_t absmax16(const float* x) {
   return fbits(r);
 }
 
-// 16 codes of x * inv (or zeros when !ok) into two words.
-__device__ __forceinline__ void enc16(const float* x, float inv, bool ok, uint32_t* w) {
+// 16 codes of x * inv (or zeros when !ok) into two words, negative zeros
+// kept (enc16_raw) or cleared (enc16).
+__device__ __forceinline__ void enc16_raw(const float* x, float inv, bool ok, uint32_t* w) {
   float v[16];
 #pragma unroll
   for (int j = 0; j < 16; j += 2) st2(v, j, __fmul2_rn(ld2(x, j), splat2(inv)));
-  w[0] = ok ? enc8_hw(v) : 0u;
-  w[1] = ok ? enc8_hw(v + 8) : 0u;
+  w[0] = ok ? enc8_raw(v) : 0u;
+  w[1] = ok ? enc8_raw(v + 8) : 0u;
+}
+__device__ __forceinline__ void enc16(const float* x, float inv, bool ok, uint32_t* w) {
+  enc16_raw(x, inv, ok, w);
+  w[0] = clear_neg_zero(w[0]);
+  w[1] = clear_neg_zero(w[1]);
 }
 
 // Signed grid values of the 8 codes of a word (element j from bits 4j..4j+3):
@@ -208,9 +223,33 @@ __device__ __forceinline__ void fwht32_lanes(float* x, int lane) {
   for (int j = 0; j < 32; j += 2) st2(x, j, __fmul2_rn(ld2(x, j), splat2(c)));
 }
 
+// Per-tensor constants of the NVFP4 scale rules, computed once per thread:
+// the tensor scale and the divisions of the group maximum by the largest
+// normalised value times it.
+struct QuantConsts {
+  float s32;
+  ExactDiv d6;   // by fp32(6 s32) (RTN, 4/6, QuEST), fp32(6 16/17 s32) (SR), 6 (MS-EDEN)
+  ExactDiv d4;   // by fp32(4 s32) (4/6)
+};
+
+template <int FMT, int RND>
+__device__ __forceinline__ QuantConsts quant_consts(uint32_t amax_in) {
+  QuantConsts c{};
+  if (FMT != FMT_NV || RND == R_AMAX) return c;
+  if (RND == R_EDEN) {
+    c.s32 = 1.0f;
+    c.d6 = exact_div_setup(FP4_EDEN_S);
+  } else {
+    c.s32 = nv_tensor_scale(amax_in, RND == R_SR ? FP4_NV_SR_DIV : FP4_NV_RTN_DIV);
+    c.d6 = exact_div_setup(__fmul_rn(c.s32, RND == R_SR ? FP4_NV_SR_GDIV : 6.0f));
+    c.d4 = exact_div_setup(__fmul_rn(c.s32, 4.0f));
+  }
+  return c;
+}
+
 template <int FMT, int RND, int HAD>
 __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t orow, int64_t ocol, int lane,
-                                              const QParams& p, const Shared& sh, uint32_t amax_in) {
+                                              const QParams& p, const Shared& sh, const QuantConsts& qc) {
   constexpr int G = FMT == FMT_NV ? 16 : 32;
   constexpr int NG = 32 / G;
   if (HAD > 0) fwht32_lanes<HAD>(x, lane);      // signs already applied by the loader
@@ -231,32 +270,33 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
   uint32_t mbits = 0;
 
   if (FMT == FMT_NV && (RND == R_RTN || RND == R_FOS || RND == R_SR || RND == R_QUEST)) {
-    const float s32 = nv_tensor_scale(amax_in, RND == R_SR ? FP4_NV_SR_DIV : FP4_NV_RTN_DIV);
+    const float s32 = qc.s32;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       const float* xg = x + 16 * g;
       const float gmax = bitsf(gmb[g]);
       uint32_t* wg = w + 2 * g;
       if (RND == R_RTN) {
-        uint32_t s8 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 6.0f)));
-        float d = __fmul_rn(e4m3_value(s8), s32), inv = __frcp_rn(d);
+        const uint32_t s8 = e4m3_rtn(exact_div(gmax, qc.d6));
+        const float d = __fmul_rn(e4m3x2_value(s8).x, s32), inv = __frcp_rn(d);
         enc16(xg, inv, finite_pos(d, inv), wg);
         sb[g] = s8;
       } else if (RND == R_FOS) {
-        uint32_t s6 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 6.0f)));
-        uint32_t s4 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 4.0f)));
-        float d6 = __fmul_rn(e4m3_value(s6), s32), i6 = __frcp_rn(d6);
-        float d4 = __fmul_rn(e4m3_value(s4), s32), i4 = __frcp_rn(d4);
+        // both candidate scales in one conversion: s6 in bits 0-7, s4 in 8-15
+        const uint32_t c2 = e4m3x2_rtn(exact_div(gmax, qc.d6), exact_div(gmax, qc.d4));
+        const float2 v2 = e4m3x2_value(c2);
+        const float d6 = __fmul_rn(v2.x, s32), i6 = __frcp_rn(d6);
+        const float d4 = __fmul_rn(v2.y, s32), i4 = __frcp_rn(d4);
         uint32_t w6[2], w4[2];
-        enc16(xg, i6, finite_pos(d6, i6), w6);
-        enc16(xg, i4, finite_pos(d4, i4), w4);
-        const bool pick4 = sse16(xg, w4, d4) < sse16(xg, w6, d6);
-        wg[0] = pick4 ? w4[0] : w6[0];
-        wg[1] = pick4 ? w4[1] : w6[1];
-        sb[g] = pick4 ? s4 : s6;
+        enc16_raw(xg, i6, finite_pos(d6, i6), w6);
+        enc16_raw(xg, i4, finite_pos(d4, i4), w4);
+        const bool pick4 = sse16(xg, w4, d4) < sse16(xg, w6, d6);   // a tie keeps the 6-scale
+        wg[0] = clear_neg_zero(pick4 ? w4[0] : w6[0]);
+        wg[1] = clear_neg_zero(pick4 ? w4[1] : w6[1]);
+        sb[g] = pick4 ? (c2 >> 8) : (c2 & 0xFFu);
       } else if (RND == R_SR) {
-        uint32_t s8 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, FP4_NV_SR_GDIV)));
-        float d = __fmul_rn(e4m3_value(s8), s32), inv = __frcp_rn(d);
+        const uint32_t s8 = e4m3_rtn(exact_div(gmax, qc.d6));
+        float d = __fmul_rn(e4m3x2_value(s8).x, s32), inv = __frcp_rn(d);
         const bool ok = finite_pos(d, inv);
         const uint64_t q0 = uint64_t(orow * p.cols + ocol + 16 * g) >> 2;
 #pragma unroll
@@ -300,7 +340,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
           }
           s8 = uint32_t(bc);
         } else {
-          s8 = e4m3_rtn(__fdiv_rn(gmax, __fmul_rn(s32, 6.0f)));
+          s8 = e4m3_rtn(exact_div(gmax, qc.d6));
         }
         float d = __fmul_rn(e4m3_value(s8), s32), inv = __frcp_rn(d);
         const bool ok = finite_pos(d, inv);
@@ -316,8 +356,8 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       const float* xg = x + 16 * g;
-      const float pq = e8m3_round(__fdiv_rn(bitsf(gmb[g]), FP4_EDEN_S));
-      const float inv = __frcp_rn(pq);
+      const float pq = e8m3_round(exact_div(bitsf(gmb[g]), qc.d6));
+      const float inv = rcp_e8m3(pq);
       enc16(xg, inv, finite_pos(pq, inv), w + 2 * g);
       float q[16], yy[16], yq[16];
       dec8(w[2 * g], q);
@@ -441,9 +481,25 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
   return lmax;
 }
 
+// Resident 256-thread blocks per SM the register allocation is held to: the
+// kernels are issue bound, and one more resident block pays for a few spilled
+// registers in RTN / amax (4 blocks) and Four-Over-Six / MS-EDEN (3 blocks);
+// SR and QuEST keep their registers.
+template <int RND>
+__host__ __device__ constexpr int quant_min_blocks() {
+  return (RND == R_RTN || RND == R_AMAX) ? 4 : ((RND == R_FOS || RND == R_EDEN) ? 3 : 1);
+}
+// The transposed kernel's shared-memory tile allows 6 blocks per SM; its
+// compute phase needs fewer registers, and 4 resident blocks overlap one
+// block's loads with the others' arithmetic.
+template <int RND>
+__host__ __device__ constexpr int quant_trans_min_blocks() {
+  return (RND == R_SR || RND == R_QUEST) ? 1 : 4;
+}
+
 // Row-wise, 32 elements per lane, grid-stride over 32-element tasks.
 template <int LOAD, int FMT, int RND, int HAD>
-__global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
+__global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QParams p) {
   __shared__ Shared sh;
   load_signs<HAD>(sh, p);
   const int lane = threadIdx.x & 31;
@@ -451,6 +507,7 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
   const uint32_t amax_in = (FMT == FMT_NV && RND != R_EDEN && RND != R_AMAX) ? *p.amax_bits : 0u;
   const float in_ts = LOAD == LD_ROW_FP4 ? *p.in_ts : 1.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) write_tensor_scale<FMT, RND>(p, amax_in);
+  const QuantConsts qc = quant_consts<FMT, RND>(amax_in);
   uint32_t acc = 0;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
   // The lane's 32 columns sit at the same offset of their rotation block on
@@ -500,7 +557,7 @@ __global__ void __launch_bounds__(256) k_quant_row32(QParams p) {
       for (int j = 0; j < 32; j += 2)
         st2(x, j, __fmul2_rn(__fmul2_rn(ld2(x, j), splat2(j < 16 ? sa : sbv)), splat2(in_ts)));
     }
-    acc = max(acc, process32<FMT, RND, HAD>(x, active, orow, ocol, lane, p, sh, amax_in));
+    acc = max(acc, process32<FMT, RND, HAD>(x, active, orow, ocol, lane, p, sh, qc));
   }
   if (RND == R_AMAX || RND == R_EDEN) block_max_atomic(acc, sh, p.amax_bits, p.status);
 }
@@ -512,7 +569,7 @@ constexpr int T32_PITCH = 144;
 __device__ __forceinline__ int t32_col(int c) { return c + 4 * (c >> 5); }
 
 template <int LOAD, int FMT, int RND, int HAD>
-__global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
+__global__ void __launch_bounds__(256, quant_trans_min_blocks<RND>()) k_quant_trans32(QParams p) {
   __shared__ Shared sh;
   __shared__ __align__(16) float tile[TR_IN_COLS][T32_PITCH];
   load_signs<HAD>(sh, p);
@@ -576,6 +633,7 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
   __syncthreads();
   const uint32_t amax_in = (FMT == FMT_NV && RND != R_EDEN && RND != R_AMAX) ? *p.amax_bits : 0u;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) write_tensor_scale<FMT, RND>(p, amax_in);
+  const QuantConsts qc = quant_consts<FMT, RND>(amax_in);
   const int orl = threadIdx.x >> 2, seg = threadIdx.x & 3;
   const int64_t orow = c0 + orl, ocol = r0 + 32 * seg;
   const bool active = orow < C && ocol < R;
@@ -585,7 +643,7 @@ __global__ void __launch_bounds__(256) k_quant_trans32(QParams p) {
     const float4 v = *reinterpret_cast<const float4*>(&tile[orl][t32_col(32 * seg) + 4 * i]);
     x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
   }
-  const uint32_t acc = process32<FMT, RND, HAD>(x, active, active ? orow : 0, active ? ocol : 0, lane, p, sh, amax_in);
+  const uint32_t acc = process32<FMT, RND, HAD>(x, active, active ? orow : 0, active ? ocol : 0, lane, p, sh, qc);
   if (RND == R_AMAX || RND == R_EDEN) block_max_atomic(acc, sh, p.amax_bits, p.status);
 }
 
@@ -618,6 +676,53 @@ static __global__ void k_selftest_e2m1(unsigned long long* mismatches) {
     }
   }
   if (bad) atomicAdd(mismatches, bad);
+}
+
+// Exhaustive and hashed checks of the exact scale shortcuts against CUDA's
+// IEEE operations; one mismatch counter each: [0] exact_div by 6 over every
+// non-negative finite fp32 dividend, [1] rcp_e8m3 over every non-negative
+// E8M3 value, [2] exact_div on 2^32 hashed (dividend, divisor) pairs over the
+// whole divisor range with quotients 2^-25 .. 2^9, [3] the E4M3 decoder over
+// every non-NaN code in both byte positions, [4] the E4M3 encoder over every
+// non-negative finite fp32 value in both byte positions.
+static __global__ void k_selftest_arith(unsigned long long* mismatches) {
+  unsigned long long bad[5] = {0, 0, 0, 0, 0};
+  const uint64_t stride = uint64_t(gridDim.x) * blockDim.x;
+  const uint64_t tid = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const ExactDiv six = exact_div_setup(6.0f);
+  for (uint64_t i = tid; i < 0x7F800000ull; i += stride) {
+    const float a = bitsf(uint32_t(i));
+    bad[0] += fbits(exact_div(a, six)) != fbits(__fdiv_rn(a, 6.0f));
+    const float t1 = bitsf(uint32_t(0x7F7FFFFFull - i));
+    const uint32_t c2 = e4m3x2_rtn(a, t1);
+    bad[4] += (c2 & 0xFFu) != e4m3_rtn(a) || (c2 >> 8) != e4m3_rtn(t1);
+  }
+  for (uint64_t i = tid; i < 255ull * 8; i += stride) {   // exponent field 0..254, 3 mantissa bits
+    const float pv = bitsf(uint32_t(((i >> 3) << 23) | ((i & 7) << 20)));
+    bad[1] += fbits(rcp_e8m3(pv)) != fbits(__frcp_rn(pv));
+  }
+  for (uint64_t i = tid; i < (1ull << 32); i += stride) {
+    const uint32_t h1 = uint32_t(i) * 0x9E3779B1u ^ uint32_t(i >> 13) * 0x85EBCA77u;
+    const uint32_t h2 = (h1 ^ (h1 >> 15)) * 0xC2B2AE3Du;
+    const uint32_t h3 = (h2 ^ (h2 >> 13)) * 0x27D4EB2Fu;
+    const int eb = 27 + int(h1 % 201u);
+    const float b = bitsf((uint32_t(eb) << 23) | (h2 & 0x7FFFFFu));
+    int ea = eb + int(h3 % 35u) - 25;
+    ea = ea < 1 ? 1 : (ea > 254 ? 254 : ea);
+    const float a = bitsf((uint32_t(ea) << 23) | (h3 >> 9));
+    const ExactDiv d = exact_div_setup(b);
+    bad[2] += fbits(exact_div(a, d)) != fbits(__fdiv_rn(a, b));
+  }
+  if (blockIdx.x == 0) {
+    for (uint32_t c = threadIdx.x; c < 127u; c += blockDim.x) {   // 0x7F is NaN, never a scale
+      const uint32_t c1 = (c * 37u + 11u) % 127u;
+      const float2 v = e4m3x2_value(c | (c1 << 8));
+      bad[3] += fbits(v.x) != fbits(e4m3_value(c)) || fbits(v.y) != fbits(e4m3_value(c1));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 5; ++k)
+    if (bad[k]) atomicAdd(mismatches + k, bad[k]);
 }
 
 }  // namespace fp4

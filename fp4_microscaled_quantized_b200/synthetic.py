@@ -74,6 +74,14 @@ def outlier_elements(shape, seed, stream=0, frac=0.001, factor=50.0):
     return f32_to_bf16_bits(x)
 
 
+def grid_values(shape, seed, stream=0, step=0.125, kmax=48):
+    """Values k * step for uniform random integers |k| <= kmax: exact in bf16
+    and so coarse that many 16-element groups have two equally good scales
+    (tie-breaking and last-bit cases)."""
+    k = rng(seed, stream).integers(-kmax, kmax + 1, size=shape)
+    return f32_to_bf16_bits((k * step).astype(np.float32))
+
+
 # ------------------------------------------------------- named workloads ----
 def linear_rtn_small(seed=0):
     """Single NVFP4 RTN forward linear: X 256x512 ~N(0,1), W 512x512 ~N(0,0.02^2)."""

@@ -99,7 +99,11 @@ typedef struct {
  * quantised tensor of rows x cols (16-byte multiple; 0 for modes without a
  * global pass).  NVFP4 RTN/QuEST/4-6/SR: one amax word.  MS-EDEN: amax, the
  * bf16 E8M3 pseudo-scales (rows * cols/16 * 2) and the fp32 EDEN factors
- * (rows * cols/block * 4) of the post hoc range alignment [QII]. */
+ * (rows * cols/block * 4) of the post hoc range alignment [QII].  Layout:
+ * the amax bits (uint32) at byte 0; the pseudo-scales, row-major, at byte
+ * 256; the EDEN factors, row-major, at byte 256 + the pseudo-scale bytes
+ * rounded up to a multiple of 256.  After an MS-EDEN call the workspace
+ * still holds these first-pass results. */
 size_t fp4_quantize_workspace_size(int64_t rows, int64_t cols, int32_t fmt,
                                    int32_t rounding, int32_t had_block);
 
@@ -263,6 +267,17 @@ unsigned long long fp4_launch_count(void);
  * ADDS the number of mismatching encoded words plus mismatching decoded
  * values to *mismatches_dev (caller zeroes it). */
 int fp4_selftest_e2m1(unsigned long long *mismatches_dev, fp4_stream_t stream);
+
+/* Device self-check of the exact shortcuts in the NVFP4 scale arithmetic
+ * against CUDA's correctly rounded division and reciprocal and the E4M3
+ * rounding.  ADDS mismatch counts to mismatches_dev[0..4] (5 counters, the
+ * caller zeroes them): [0] the corrected division by 6 over every
+ * non-negative finite fp32 dividend, [1] the reciprocal of every
+ * non-negative E8M3 value, [2] the corrected division by a per-tensor
+ * divisor on 2^32 hashed dividend/divisor pairs, [3] the hardware E4M3
+ * decoder over every non-NaN code, [4] the hardware E4M3 encoder over every
+ * non-negative finite fp32 value. */
+int fp4_selftest_arith(unsigned long long *mismatches_dev, fp4_stream_t stream);
 
 /* Static description of a status code. */
 const char *fp4_status_string(int status);

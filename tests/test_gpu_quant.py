@@ -132,6 +132,14 @@ def test_hardware_e2m1_encoder_exhaustive(cuda_lib):
     assert cuda_lib.selftest_e2m1() == 0
 
 
+def test_exact_scale_arithmetic(cuda_lib):
+    """The corrected divisions and the E8M3 reciprocal of the NVFP4 scale
+    path equal CUDA's correctly rounded __fdiv_rn / __frcp_rn on every case
+    checked, and the hardware E4M3 conversions equal the scale rounding and
+    the code table."""
+    assert cuda_lib.selftest_arith() == [0, 0, 0, 0, 0]
+
+
 @pytest.mark.parametrize("fmt,rnd,had", [(qn.NVFP4, qn.FOUR_OVER_SIX, 0), (qn.NVFP4, qn.MS_EDEN, 16),
                                          (qn.NVFP4, qn.SR, 16), (qn.NVFP4, qn.QUEST, 0)])
 @pytest.mark.parametrize("transpose", [False, True])
@@ -151,3 +159,42 @@ def test_launch_counter_counts_kernels(cuda_lib):
     cuda_lib.quantize(x, qn.NVFP4, qn.MS_EDEN, 128, randomized=True)      # pass 1 + pass 2
     cuda_lib.quantize(x, qn.NVFP4, qn.FOUR_OVER_SIX, 0)                     # amax + quantise
     assert cuda_lib.launch_count() - n0 == 4
+
+
+@pytest.mark.parametrize("had,transpose", [(0, False), (0, True), (16, False), (128, True)])
+def test_four_over_six_grid_ties(cuda_lib, had, transpose):
+    """Four-Over-Six on a coarse value grid, where many groups' two candidate
+    errors tie exactly or within an ulp: a single product, difference or sum
+    of the squared-error evaluation rounded differently flips a pick."""
+    bits = syn.grid_values((512, 2048), seed=11, stream=had)
+    x = syn.bf16_bits_to_f32(bits)
+    g = cuda_lib.quantize(to_dev(bits), qn.NVFP4, qn.FOUR_OVER_SIX, had, transpose=transpose)
+    o = qn.quantize(x, qn.NVFP4, qn.FOUR_OVER_SIX, had, transpose=transpose)
+    assert_qt_equal(g, o)
+
+
+@pytest.mark.parametrize("had,transpose", [(128, False), (128, True), (16, False), (32, True)])
+def test_ms_eden_first_pass_bit_exact(cuda_lib, had, transpose):
+    """MS-EDEN's first-pass results in the workspace -- the bf16 pseudo-scales
+    and the EDEN factors S = <y,y> / <y,q p> -- equal the oracle's bit for bit.
+    S is a ratio of two fp32 pairwise sums, so this pins every product and
+    the order of every sum, which the final scales (a stochastic rounding of
+    S p) would show only rarely."""
+    shape = (384, 1024)
+    bits = syn.student_t(shape, seed=5, stream=had, unit_rms=True)
+    x = syn.bf16_bits_to_f32(bits)
+    rows, cols = (shape[1], shape[0]) if transpose else shape
+    ws = cuda_lib.alloc_workspace(cuda_lib.workspace_size(rows, cols, qn.NVFP4, qn.MS_EDEN, had))
+    seed = 0xC0FFEE
+    g = cuda_lib.quantize(to_dev(bits), qn.NVFP4, qn.MS_EDEN, had, randomized=True, seed=seed, sign_tag=1,
+                          tensor_tag=2, transpose=transpose, ws=ws)
+    o = qn.quantize(x, qn.NVFP4, qn.MS_EDEN, had, True, seed, 1, 2, transpose=transpose)
+    torch.cuda.synchronize()
+    wsb = ws.cpu().numpy()
+    n_pseudo = rows * (cols // 16) * 2
+    pseudo = wsb[256:256 + n_pseudo].view(np.uint16).reshape(rows, cols // 16)
+    s_off = 256 + (n_pseudo + 255) // 256 * 256
+    S = wsb[s_off:s_off + rows * (cols // had) * 4].view(np.uint32).reshape(rows, cols // had)
+    np.testing.assert_array_equal(pseudo, (o.extra["pseudo"].view(np.uint32) >> 16).astype(np.uint16))
+    np.testing.assert_array_equal(S, o.extra["S"].view(np.uint32))
+    assert_qt_equal(g, o)
