@@ -61,6 +61,7 @@ struct Params {
   void* D;
   const uint8_t* mask;  // epilogue clip mask (M x N bits) or null
   int* status;
+  int raster;           // CTA-pair tile order (tile_coords2)
 };
 
 // ----------------------------------------------------------- PTX helpers --
@@ -608,12 +609,25 @@ __device__ __forceinline__ void mma_pair(uint32_t d, uint64_t a, uint64_t b, uin
   }
 }
 
-// Pair tile order: groups of 8 256-row blocks sweep all 256-column blocks.
-__device__ __forceinline__ void tile_coords2(int64_t t, int64_t nm, int64_t nn, int64_t& mb, int64_t& nb) {
-  const int64_t G = 8;
-  int64_t per_group = G * nn;
-  int64_t g = t / per_group, r = t % per_group;
-  int64_t gm = nm - g * G < G ? nm - g * G : G;
+// Pair tile order.  raster > 0: groups of `raster` 256-row blocks sweep all
+// 256-column blocks (each B tile is fetched once per group and shared by the
+// group's tiles of one wave); raster < 0: groups of -raster column blocks
+// sweep all row blocks (the same with A and B exchanged).
+__device__ __forceinline__ void tile_coords2(int64_t t, int64_t nm, int64_t nn, int raster, int64_t& mb,
+                                             int64_t& nb) {
+  if (raster < 0) {
+    const int64_t G = -raster;
+    const int64_t per_group = G * nm;
+    const int64_t g = t / per_group, r = t % per_group;
+    const int64_t gn = nn - g * G < G ? nn - g * G : G;
+    nb = g * G + r % gn;
+    mb = r / gn;
+    return;
+  }
+  const int64_t G = raster;
+  const int64_t per_group = G * nn;
+  const int64_t g = t / per_group, r = t % per_group;
+  const int64_t gm = nm - g * G < G ? nm - g * G : G;
   mb = g * G + r % gm;
   nb = r / gm;
 }
@@ -685,7 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     const int64_t nrb_a = (p.M + 127) / 128, nrb_b = (p.N + 127) / 128;
     for (int64_t t = pair_id; t < ntiles && !*abort_flag; t += npairs) {
       int64_t mb, nb;
-      tile_coords2(t, nm, nn, mb, nb);
+      tile_coords2(t, nm, nn, p.raster, mb, nb);
       const int64_t ra = mb * 2 + rank, rb = nb * 2 + rank;          // this CTA's 128-row blocks
       // 128-row halves that exist (a half entirely past M or N is not loaded)
       const int a_halves = (mb * 2 + 1 < nrb_a) ? 2 : 1, b_halves = (nb * 2 + 1 < nrb_b) ? 2 : 1;
@@ -818,7 +832,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     const float tscale = __fmul_rn(*p.ta, *p.tb);
     for (int64_t t = pair_id; t < ntiles; t += npairs) {
       int64_t mb, nb;
-      tile_coords2(t, nm, nn, mb, nb);
+      tile_coords2(t, nm, nn, p.raster, mb, nb);
       const bool got = wait_c(acc_full, acc_ph, abort_flag, p.status);
       uint32_t bad;
       asm volatile(
@@ -1048,6 +1062,10 @@ extern "C" int fp4_gemm(const fp4_qtensor* A, const fp4_qtensor* B, void* D, int
   p.nkb = (K / (A->fmt == FP4_NVFP4 ? 16 : 32) + 3) / 4;
   p.ta = A->tensor_scale; p.tb = B->tensor_scale;
   p.D = D; p.mask = epi_mask; p.status = status_ptr();
+  // Tile order of the pair kernel (measured on the Llama-shaped layer set):
+  // with at least as many rows as columns, groups of 8 column blocks sweep
+  // the rows; otherwise groups of 16 row blocks sweep the columns.
+  p.raster = M >= N ? -8 : 16;
   cudaError_t e;
   const bool nv = A->fmt == FP4_NVFP4, bf = out_dtype == 1, epi = epi_inverse_had == 32;
 #define FP4_GEMM_LAUNCH(F, O, E) \
