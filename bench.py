@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--sweep-cases", default="all",
                     help="comma list of sweep case names (e.g. nvfp4-fos-h0,nvfp4-eden-h128) or 'all'")
     ap.add_argument("--sweep-reps", type=int, default=10)
+    ap.add_argument("--diagnostics", action="store_true",
+                    help="quantisation MSE (Table 1) and projection magnitude misalignment of every "
+                         "mode, computed with the library's kernels; one JSON line per case")
     args = ap.parse_args()
     global LAYERS
     keep = args.layers.split(",")
@@ -507,6 +510,13 @@ def main():
     if args.quant_sweep:
         if rank == 0:
             quant_sweep(args)
+        return
+    if args.diagnostics:
+        if rank == 0:
+            from fp4_microscaled_quantized_b200 import api, diagnostics
+            api.load()
+            for row in diagnostics.table(torch.device("cuda", local)):
+                print(json.dumps(row), flush=True)
         return
     from fp4_microscaled_quantized_b200 import api
     api.load()

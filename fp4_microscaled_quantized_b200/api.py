@@ -216,6 +216,21 @@ def requantize(qt, rnd, had_block=0, randomized=False, seed=0, sign_tag=0, tenso
     return out
 
 
+def dequantize(qt, out_dtype=torch.float32, out=None):
+    """fp4_dequantize: the fp32 (or bf16) value of every element of a
+    quantised tensor (needs its linear scales)."""
+    lib = load()
+    f = lib.fp4_dequantize
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(fp4_qtensor), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
+    if out is None:
+        out = torch.empty((qt.rows, qt.cols), dtype=out_dtype, device=qt.codes.device)
+    code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
+    cs = qt.c_struct()
+    _check(f(ctypes.byref(cs), _ptr(out), code, _stream()), "fp4_dequantize")
+    return out
+
+
 def hadamard(x, block, randomized=False, seed=0, sign_tag=0):
     lib = load()
     y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
@@ -247,7 +262,7 @@ def gemm(A, B, out_dtype=torch.float32, mask=None, inverse_had=0, out=None):
     return out
 
 
-RECIPE_QUARTET, RECIPE_QUARTET2, RECIPE_RTN = 0, 1, 2
+RECIPE_QUARTET, RECIPE_QUARTET2, RECIPE_RTN, RECIPE_TETRAJET2 = 0, 1, 2, 3
 
 
 class fp4_recipe(ctypes.Structure):

@@ -85,6 +85,39 @@ __global__ void k_swizzle(const uint8_t* sc, int64_t rows, int64_t ng, int64_t n
     swz[swz_offset(i / ng, i % ng, nkb)] = sc[i];
 }
 
+// De-quantisation: 8 elements (one 32-bit code word, inside one scale group)
+// per task, fp32(fp32(q * s_group) * s_tensor), written as fp32 or bf16.
+template <int OUT>
+__global__ void __launch_bounds__(256) k_dequant(const uint8_t* codes, const uint8_t* scales, const float* ts,
+                                                 int fmt, int64_t rows, int64_t cols, void* D) {
+  const int64_t words_per_row = cols >> 3, n = rows * words_per_row;
+  const int gsh = fmt == FP4_NVFP4 ? 4 : 5;
+  const float t = *ts;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / words_per_row, c = (i - r * words_per_row) << 3;
+    const uint32_t w = reinterpret_cast<const uint32_t*>(codes)[i];
+    const uint32_t sc = scales[r * (cols >> gsh) + (c >> gsh)];
+    const float sg = fmt == FP4_NVFP4 ? e4m3_value(sc) : pow2f(int(sc) - 127);
+    float q[8];
+    dec8(w, q);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) q[j] = __fmul_rn(__fmul_rn(q[j], sg), t);
+    if (OUT == 0) {
+      float4* d = reinterpret_cast<float4*>(static_cast<float*>(D) + (i << 3));
+      d[0] = make_float4(q[0], q[1], q[2], q[3]);
+      d[1] = make_float4(q[4], q[5], q[6], q[7]);
+    } else {
+      uint32_t h[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(q[2 * j], q[2 * j + 1]);
+        h[j] = *reinterpret_cast<const uint32_t*>(&b);
+      }
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(D) + (i << 3)) = make_uint4(h[0], h[1], h[2], h[3]);
+    }
+  }
+}
+
 static int launch_pad(uint8_t* swz, int64_t rows, int64_t ng, cudaStream_t s) {
   int64_t nkb = (ng + 3) / 4;
   if (!swz || ((rows % 128) == 0 && (ng % 4) == 0)) return FP4_OK;
@@ -213,6 +246,26 @@ int fp4_requantize(const fp4_qtensor* in, int32_t transpose, int32_t rounding, f
   p.randomized = had.randomized ? 1 : 0;
   return run_quant(transpose ? LD_TRANS_FP4 : LD_ROW_FP4, fmt, rounding, had.block, p, ws,
                    ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fp4_dequantize(const fp4_qtensor* in, void* D, int32_t out_dtype, fp4_stream_t stream) {
+  if (!in || (in->fmt != FP4_MXFP4 && in->fmt != FP4_NVFP4) || (out_dtype != 0 && out_dtype != 1))
+    return FP4_ERR_INVALID_ARG;
+  const int g = in->fmt == FP4_NVFP4 ? 16 : 32;
+  if (in->rows < 0 || in->cols < 0 || in->cols % g) return FP4_ERR_INVALID_ARG;
+  if (in->rows == 0 || in->cols == 0) return FP4_OK;
+  if (!in->codes || !in->scales || !in->tensor_scale || !D) return FP4_ERR_INVALID_ARG;
+  if (!aligned(in->codes, 16) || !aligned(D, 16) || !aligned(in->tensor_scale, 4)) return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = in->rows * (in->cols >> 3);
+  int64_t blocks = (n + 255) / 256, cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (out_dtype == 0)
+    k_dequant<0><<<unsigned(blocks), 256, 0, s>>>(in->codes, in->scales, in->tensor_scale, in->fmt, in->rows, in->cols, D);
+  else
+    k_dequant<1><<<unsigned(blocks), 256, 0, s>>>(in->codes, in->scales, in->tensor_scale, in->fmt, in->rows, in->cols, D);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
 }
 
 int fp4_hadamard(const void* x, float* y, int64_t rows, int64_t cols, fp4_had had, uint64_t seed,

@@ -77,6 +77,9 @@ int fp4_recipe_preset(int32_t id, fp4_recipe* r) {
     case FP4_RECIPE_RTN:
       *r = fp4_recipe{FP4_NVFP4, FP4_RTN, 0, FP4_RTN, 0, 0, 0, 0, 0, 0};
       return FP4_OK;
+    case FP4_RECIPE_TETRAJET2:
+      *r = fp4_recipe{FP4_NVFP4, FP4_RTN, 0, FP4_SR, 128, 1, 0, 0, 0, 0};
+      return FP4_OK;
     default:
       return FP4_ERR_INVALID_ARG;
   }

@@ -107,6 +107,19 @@ typedef struct {
 size_t fp4_quantize_workspace_size(int64_t rows, int64_t cols, int32_t fmt,
                                    int32_t rounding, int32_t had_block);
 
+/* De-quantise a quantised tensor: D[r][c] = fp32(fp32(q * s_group) * s_tensor)
+ * for the E2M1 value q of element (r, c), its group's scale s_group (E4M3 for
+ * NVFP4, 2^(e-127) for MXFP4, from the LINEAR scales) and the tensor scale --
+ * the dequantised value x_FP4 * x_FP8 * x_FP32 of [QII] "NVFP4 Format and
+ * Standard Stochastic Rounding", rounded as the backward re-quantisation
+ * reads a saved tensor ([QII] "The Complete Quartet II Computation Graph").
+ * D_dev: rows x cols row-major, fp32 (out_dtype 0) or bf16 rounded to nearest
+ * even (1), caller-owned, 16-byte aligned.  in: codes (16-byte aligned),
+ * scales and tensor_scale required.  Asynchronous on `stream`; an empty tensor
+ * launches nothing.  Errors: FP4_ERR_INVALID_ARG (null pointers, format,
+ * out_dtype, cols not a multiple of the group), FP4_ERR_ALIGNMENT. */
+int fp4_dequantize(const fp4_qtensor *in, void *D_dev, int32_t out_dtype, fp4_stream_t stream);
+
 /* Bytes of the swizzled scale buffer for rows x n_groups scales. */
 size_t fp4_swizzled_scale_bytes(int64_t rows, int64_t n_groups);
 
@@ -206,10 +219,21 @@ int fp4_gemm(const fp4_qtensor *A, const fp4_qtensor *B, void *D_dev, int32_t ou
  *      Four-Over-Six, no rotation; backward de-quantise, transpose, RHT128 on
  *      the inner dimension, MS-EDEN; no inverse transform.
  *  FP4_RECIPE_RTN      NVFP4 RTN on every operand, no rotation.
+ *  FP4_RECIPE_TETRAJET2 the simplified (GPU-feasible) TetraJet-v2 the [QII]
+ *      page compares against ("Comparison to TetraJet-v2 and the NVIDIA
+ *      recipe"): NVFP4; forward RTN with native 1x16 scales, no rotation;
+ *      backward de-quantise, transpose, RHT128 on the inner dimension and
+ *      element-wise SR (the same graph as FP4_RECIPE_QUARTET2 with SR in
+ *      place of MS-EDEN).
  * Seeds: every random draw of one backward step is keyed by step_seed; the
  * dX GEMM's operands share sign tag 0, the dW GEMM's sign tag 1; SR tensor
  * tags 1 (dY), 2 (W_q^T), 3 (dY^T), 4 (X_q^T); forward tags 5 (X), 6 (W). */
-enum fp4_recipe_id { FP4_RECIPE_QUARTET = 0, FP4_RECIPE_QUARTET2 = 1, FP4_RECIPE_RTN = 2 };
+enum fp4_recipe_id {
+  FP4_RECIPE_QUARTET = 0,
+  FP4_RECIPE_QUARTET2 = 1,
+  FP4_RECIPE_RTN = 2,
+  FP4_RECIPE_TETRAJET2 = 3
+};
 
 typedef struct {
   int32_t fmt;            /* fp4_format of every operand                     */

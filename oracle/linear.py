@@ -12,6 +12,12 @@ Test infrastructure only (see ``oracle/__init__.py``).
   transpose, RHT128 on the inner dimension and MS-EDEN for (E, W^T) and
   (E^T, X^T); no inverse transform.
 * RTN -- a single NVFP4 RTN linear layer without rotation.
+* TETRAJET2 -- the simplified TetraJet-v2 of the Quartet II page ("Comparison
+  to TetraJet-v2 and the NVIDIA recipe"): NVFP4 RTN with native 1x16 scales
+  on the forward pass, SR with the RHT on the inner dimension for both
+  backward GEMMs, weights and activations re-quantised -- the QUARTET2 graph
+  with SR in place of MS-EDEN (READING: the same 128-element rotation, since
+  the page names MS-EDEN as the one difference).
 
 READING (seed scheme, the pages name none): every random draw of one
 backward step uses key = step_seed; the two GEMMs' rotations use sign tags
@@ -44,6 +50,7 @@ class Recipe:
 QUARTET = Recipe(qn.MXFP4, qn.QUEST, 32, qn.SR, 32, True, True)
 QUARTET2 = Recipe(qn.NVFP4, qn.FOUR_OVER_SIX, 0, qn.MS_EDEN, 128, True, False)
 RTN = Recipe(qn.NVFP4, qn.RTN, 0, qn.RTN, 0, False, False)
+TETRAJET2 = Recipe(qn.NVFP4, qn.RTN, 0, qn.SR, 128, True, False)
 
 
 def linear_fwd(X, W, r, seed=0):

@@ -1,5 +1,6 @@
 """Pins of the oracle GEMM reference and linear-layer recipes."""
 import numpy as np
+import pytest
 
 from fp4_microscaled_quantized_b200 import synthetic as syn
 from oracle import gemm as gm
@@ -70,11 +71,12 @@ def test_quartet_forward_and_backward_track_exact_gradients():
     assert float(ops["E_row"].tensor_scale) * float(ops["W_t"].tensor_scale) == np.float32(4 / 3) ** 2
 
 
-def test_quartet2_backward_is_unbiased_in_the_mean():
+@pytest.mark.parametrize("recipe", [ln.QUARTET2, ln.TETRAJET2], ids=["quartet2", "tetrajet2"])
+def test_quartet2_backward_is_unbiased_in_the_mean(recipe):
     M, N, K = 128, 128, 256
     d = syn.linear_quartet2(M, N, K, 4)
     X, W, dY = (syn.bf16_bits_to_f32(d[k]) for k in ("X", "W", "dY"))
-    _, _, ctx = ln.linear_fwd(X, W, ln.QUARTET2)
+    _, _, ctx = ln.linear_fwd(X, W, recipe)
     # target: the product with the saved (forward-quantised) operands
     wq = qn.dequant_f64(ctx["Wq"])
     xq = qn.dequant_f64(ctx["Xq"])
@@ -85,7 +87,7 @@ def test_quartet2_backward_is_unbiased_in_the_mean():
     n = 16
     single = None
     for s in range(n):
-        (dx, _), (dw, _), _ = ln.linear_bwd(dY, ctx, ln.QUARTET2, step_seed=s)
+        (dx, _), (dw, _), _ = ln.linear_bwd(dY, ctx, recipe, step_seed=s)
         acc_dx += dx
         acc_dw += dw
         if single is None:
@@ -117,3 +119,25 @@ def test_epilogue_bound_propagation():
         for blk in range(2):
             sl = slice(32 * blk, 32 * blk + 32)
             np.testing.assert_allclose(ob[r, sl], h @ (bound[r, sl] * keep[r, sl]))
+
+
+def test_ms_eden_backward_beats_sr_backward():
+    """The Quartet II page's comparison with the simplified TetraJet-v2: the
+    same backward graph with MS-EDEN in place of SR estimates both gradients
+    with less error (per-tensor MSE more than 2x lower, "Table 1"; Figure 1)."""
+    M, N, K = 256, 256, 512
+    d = syn.linear_quartet2(M, N, K, 6)
+    X, W, dY = (syn.bf16_bits_to_f32(d[k]) for k in ("X", "W", "dY"))
+    err = {}
+    for name, r in (("eden", ln.QUARTET2), ("sr", ln.TETRAJET2)):
+        _, _, ctx = ln.linear_fwd(X, W, r)
+        tgt_dx = dY.astype(np.float64) @ qn.dequant_f64(ctx["Wq"])
+        tgt_dw = dY.astype(np.float64).T @ qn.dequant_f64(ctx["Xq"])
+        e = [0.0, 0.0]
+        for s in range(4):
+            (dx, _), (dw, _), _ = ln.linear_bwd(dY, ctx, r, step_seed=s)
+            e[0] += np.sum((dx - tgt_dx) ** 2)
+            e[1] += np.sum((dw - tgt_dw) ** 2)
+        err[name] = e
+    assert err["eden"][0] < 0.7 * err["sr"][0]
+    assert err["eden"][1] < 0.7 * err["sr"][1]
