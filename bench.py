@@ -348,14 +348,14 @@ RND_NAMES = {0: "rtn", 1: "quest", 2: "fos", 3: "sr", 4: "eden"}
 def sweep_cases(api):
     """(name, fmt, rounding, had_block, randomized) of every combination the C ABI
     accepts: MXFP4 (RTN, QuEST, SR) and NVFP4 (RTN, QuEST, 4/6, SR) with Hadamard
-    none/16/32/128, NVFP4 MS-EDEN with 16/32/128.  The stochastic modes use the
+    none/16/32/64/128/256, NVFP4 MS-EDEN with 16/32/64/128/256.  The stochastic modes use the
     randomized transform (backward pass), the others the deterministic one."""
     out = []
     for fmt, fname, rnds in ((api.MXFP4, "mxfp4", (api.RTN, api.QUEST, api.SR)),
                              (api.NVFP4, "nvfp4", (api.RTN, api.QUEST, api.FOUR_OVER_SIX, api.SR,
                                                    api.MS_EDEN))):
         for rnd in rnds:
-            for had in (0, 16, 32, 128):
+            for had in (0, 16, 32, 64, 128, 256):
                 if rnd == api.MS_EDEN and had == 0:
                     continue
                 rand = rnd in (api.SR, api.MS_EDEN) and had > 0

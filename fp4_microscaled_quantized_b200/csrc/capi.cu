@@ -62,7 +62,7 @@ static WsLayout ws_layout(int64_t rows, int64_t cols, int fmt, int rnd, int had)
 }
 
 static bool combo_supported(int fmt, int rnd, int had) {
-  if (had != 0 && had != 16 && had != 32 && had != 128) return false;
+  if (had != 0 && had != 16 && had != 32 && had != 64 && had != 128 && had != 256) return false;
   if (fmt == FP4_MXFP4 && (rnd == FP4_FOUR_OVER_SIX || rnd == FP4_MS_EDEN)) return false;
   int g = fmt == FP4_NVFP4 ? 16 : 32;
   if (rnd == FP4_MS_EDEN && (had == 0 || had < g)) return false;
@@ -163,7 +163,9 @@ static int run_quant(int load, int fmt, int rnd, int had, QParams& p, void* ws, 
     switch (had) {
       case 16: k_eden_pass2<16><<<unsigned(blocks), 256, 0, s>>>(p); break;
       case 32: k_eden_pass2<32><<<unsigned(blocks), 256, 0, s>>>(p); break;
-      default: k_eden_pass2<128><<<unsigned(blocks), 256, 0, s>>>(p); break;
+      case 64: k_eden_pass2<64><<<unsigned(blocks), 256, 0, s>>>(p); break;
+      case 128: k_eden_pass2<128><<<unsigned(blocks), 256, 0, s>>>(p); break;
+      default: k_eden_pass2<256><<<unsigned(blocks), 256, 0, s>>>(p); break;
     }
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
@@ -202,6 +204,7 @@ int fp4_quantize(const void* x, int64_t in_rows, int64_t in_cols, int32_t transp
   const int64_t chunk = had.block > g ? had.block : g;
   if (cols % chunk) return FP4_ERR_INVALID_ARG;
   if (transpose && (in_cols % 8)) return FP4_ERR_ALIGNMENT;
+  if (transpose && had.block > 128) return FP4_ERR_UNSUPPORTED;   // longer than the transposed tile
   out->rows = rows; out->cols = cols; out->fmt = fmt;
   if (rows == 0 || cols == 0) return FP4_OK;   // empty tensor: nothing to launch
   int st = check_out(out);
@@ -233,6 +236,7 @@ int fp4_requantize(const fp4_qtensor* in, int32_t transpose, int32_t rounding, f
   const int64_t chunk = had.block > g ? had.block : g;
   if (cols % chunk) return FP4_ERR_INVALID_ARG;
   if (transpose && (in->cols % 16)) return FP4_ERR_ALIGNMENT;
+  if (transpose && had.block > 128) return FP4_ERR_UNSUPPORTED;   // longer than the transposed tile
   out->rows = rows; out->cols = cols; out->fmt = fmt;
   if (rows == 0 || cols == 0) return FP4_OK;
   int st = check_out(out);
@@ -270,7 +274,8 @@ int fp4_dequantize(const fp4_qtensor* in, void* D, int32_t out_dtype, fp4_stream
 
 int fp4_hadamard(const void* x, float* y, int64_t rows, int64_t cols, fp4_had had, uint64_t seed,
                  fp4_stream_t stream) {
-  if (had.block != 16 && had.block != 32 && had.block != 128) return FP4_ERR_UNSUPPORTED;
+  if (had.block != 16 && had.block != 32 && had.block != 64 && had.block != 128 && had.block != 256)
+    return FP4_ERR_UNSUPPORTED;
   if (rows < 0 || cols < 0 || cols % had.block) return FP4_ERR_INVALID_ARG;
   if (rows == 0 || cols == 0) return FP4_OK;
   if (!x || !y) return FP4_ERR_INVALID_ARG;
@@ -284,7 +289,9 @@ int fp4_hadamard(const void* x, float* y, int64_t rows, int64_t cols, fp4_had ha
   switch (had.block) {
     case 16: k_hadamard<16><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
     case 32: k_hadamard<32><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
-    default: k_hadamard<128><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
+    case 64: k_hadamard<64><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
+    case 128: k_hadamard<128><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
+    default: k_hadamard<256><<<unsigned(blocks), 256, 0, s>>>(p, y); break;
   }
   count_launch();
   return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;

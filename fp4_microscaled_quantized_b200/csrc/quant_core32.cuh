@@ -185,7 +185,7 @@ __device__ __forceinline__ uint32_t lane_signs(const Shared& sh, const QParams& 
 }
 
 // Block FWHT over HAD consecutive elements, 32 per lane (HAD / 32 aligned
-// lanes for HAD = 128), same butterfly order as fwht8_lanes.  The random
+// lanes for HAD = 64, 128, 256), same butterfly order as fwht8_lanes.  The random
 // signs are applied by the loaders (to the bf16 bits or the FP4 codes).  The
 // h = 1 stage works inside the natural pairs (2i, 2i+1); every later stage,
 // the cross-lane ones (x + o on the lower lane, o - x on the upper: one
@@ -218,7 +218,7 @@ __device__ __forceinline__ void fwht32_lanes(float* x, int lane) {
       st2(x, i, __ffma2_rn(sgn, ld2(x, i), o));
     }
   }
-  const float c = HAD == 16 ? 0.25f : (HAD == 32 ? 0.176776695296636881f : 0.0883883476483184405f);
+  const float c = hadamard_scale<HAD>();
 #pragma unroll
   for (int j = 0; j < 32; j += 2) st2(x, j, __fmul2_rn(ld2(x, j), splat2(c)));
 }
@@ -382,12 +382,12 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
       if (active) *reinterpret_cast<float2*>(p.eden_S + orow * (p.cols >> 4) + (ocol >> 4)) = make_float2(S2[0], S2[1]);
     } else {
       float num = __fadd_rn(num_g[0], num_g[NG - 1]), den = __fadd_rn(den_g[0], den_g[NG - 1]);
-      if (HAD == 128) {
-        num = tree_lanes<4>(num);
-        den = tree_lanes<4>(den);
+      if (HAD > 32) {                      // the block spans HAD / 32 aligned lanes
+        num = tree_lanes<(HAD > 32 ? HAD / 32 : 1)>(num);
+        den = tree_lanes<(HAD > 32 ? HAD / 32 : 1)>(den);
       }
       const float S = den > 0.0f ? __fdiv_rn(num, den) : 1.0f;
-      if (active && (HAD == 32 || (lane & 3) == 0)) p.eden_S[orow * (p.cols / HAD) + ocol / HAD] = S;
+      if (active && (lane & (HAD > 32 ? HAD / 32 - 1 : 0)) == 0) p.eden_S[orow * (p.cols / HAD) + ocol / HAD] = S;
     }
   } else if (FMT == FMT_MX && (RND == R_RTN || RND == R_SR)) {
     int e = int(gmb[0] >> 23) - 129;
@@ -513,7 +513,7 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
   // The lane's 32 columns sit at the same offset of their rotation block on
   // every task (cols is a multiple of the block, the stride of 32 tasks), so
   // its sign masks are fixed for the whole loop.
-  const uint32_t sw = lane_signs<HAD>(sh, p, 32 * (lane & 3));
+  const uint32_t sw = lane_signs<HAD>(sh, p, 32 * (lane & 7));
   uint32_t sm[LOAD == LD_ROW ? 16 : 4];
   if (LOAD == LD_ROW) sign_masks_bf16(sw, sm);
   else sign_masks_fp4(sw, sm);

@@ -31,35 +31,46 @@ int resident_blocks() {
 
 template <int LOAD, int FMT, int RND, int HAD>
 cudaError_t launch_one(const QParams& p, cudaStream_t s) {
-  const bool wide = (p.cols % 32) == 0;   // 32 elements per lane
-  if ((LOAD == LD_ROW || LOAD == LD_ROW_FP4) && wide) {
-    int64_t tasks = p.rows * (p.cols >> 5);
-    int64_t blocks = (tasks + 255) / 256;
-    int64_t cap = int64_t(num_sms()) * resident_blocks<true, LOAD, FMT, RND, HAD>();
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    k_quant_row32<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
-    count_launch();
-  } else if (wide) {
-    dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
-              unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
-    k_quant_trans32<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
-    count_launch();
-  } else if (LOAD == LD_ROW || LOAD == LD_ROW_FP4) {
-    int64_t tasks = p.rows * (p.cols >> 3);
-    int64_t blocks = (tasks + 255) / 256;
-    int64_t cap = int64_t(num_sms()) * resident_blocks<false, LOAD, FMT, RND, HAD>();
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    k_quant_row<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
-    count_launch();
+  constexpr bool TRANS = LOAD == LD_TRANS || LOAD == LD_TRANS_FP4;
+  if constexpr (TRANS && HAD > 128) {
+    // a rotation block longer than the transposed kernel's 128-row tile
+    return cudaErrorInvalidValue;
   } else {
-    dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
-              unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
-    k_quant_trans<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
-    count_launch();
+    const bool wide = (p.cols % 32) == 0;   // 32 elements per lane (always so for blocks >= 32)
+    if (!TRANS && wide) {
+      int64_t tasks = p.rows * (p.cols >> 5);
+      int64_t blocks = (tasks + 255) / 256;
+      int64_t cap = int64_t(num_sms()) * resident_blocks<true, LOAD, FMT, RND, HAD>();
+      if (blocks > cap) blocks = cap;
+      if (blocks < 1) blocks = 1;
+      k_quant_row32<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
+      count_launch();
+    } else if (wide) {
+      dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
+                unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
+      k_quant_trans32<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
+      count_launch();
+    } else if constexpr (HAD <= 16) {
+      // inner dimension 16 mod 32: 8 elements per lane
+      if (!TRANS) {
+        int64_t tasks = p.rows * (p.cols >> 3);
+        int64_t blocks = (tasks + 255) / 256;
+        int64_t cap = int64_t(num_sms()) * resident_blocks<false, LOAD, FMT, RND, HAD>();
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+        k_quant_row<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
+        count_launch();
+      } else {
+        dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
+                  unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
+        k_quant_trans<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
+        count_launch();
+      }
+    } else {
+      return cudaErrorInvalidValue;          // cols is a multiple of the block: unreachable
+    }
+    return cudaGetLastError();
   }
-  return cudaGetLastError();
 }
 
 #define FP4_HAD_SWITCH(LOAD, FMT, RND)                                      \
@@ -67,7 +78,9 @@ cudaError_t launch_one(const QParams& p, cudaStream_t s) {
     case 0: return launch_one<LOAD, FMT, RND, 0>(p, s);                     \
     case 16: return launch_one<LOAD, FMT, RND, 16>(p, s);                   \
     case 32: return launch_one<LOAD, FMT, RND, 32>(p, s);                   \
+    case 64: return launch_one<LOAD, FMT, RND, 64>(p, s);                   \
     case 128: return launch_one<LOAD, FMT, RND, 128>(p, s);                 \
+    case 256: return launch_one<LOAD, FMT, RND, 256>(p, s);                 \
     default: return cudaErrorInvalidValue;                                  \
   }
 
@@ -75,7 +88,9 @@ cudaError_t launch_one(const QParams& p, cudaStream_t s) {
   switch (had) {                                                            \
     case 16: return launch_one<LOAD, FMT, RND, 16>(p, s);                   \
     case 32: return launch_one<LOAD, FMT, RND, 32>(p, s);                   \
+    case 64: return launch_one<LOAD, FMT, RND, 64>(p, s);                   \
     case 128: return launch_one<LOAD, FMT, RND, 128>(p, s);                 \
+    case 256: return launch_one<LOAD, FMT, RND, 256>(p, s);                 \
     default: return cudaErrorInvalidValue;                                  \
   }
 

@@ -106,7 +106,7 @@ __device__ __forceinline__ void encode_rtn8(const float* x, float inv, bool ok, 
 }
 
 struct Shared {
-  uint32_t signs[4];   // RHT sign bits of one rotation block (<= 128)
+  uint32_t signs[8];   // RHT sign bits of one rotation block (<= 256)
   uint32_t red[32];    // block reductions
 };
 
@@ -312,7 +312,7 @@ __device__ __forceinline__ uint32_t process8(float* x, bool active, int64_t orow
 // Fill the random sign bits of one rotation block into shared memory.
 template <int HAD>
 __device__ __forceinline__ void load_signs(Shared& sh, const QParams& p) {
-  if (threadIdx.x < 4) sh.signs[threadIdx.x] = 0;
+  if (threadIdx.x < 8) sh.signs[threadIdx.x] = 0;
   __syncthreads();
   if (HAD > 0 && p.randomized && threadIdx.x < HAD / 4) {
     u32x4 b = philox_block(p.seed, threadIdx.x, TAG_RHT_SIGN, p.sign_tag);

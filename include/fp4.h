@@ -71,7 +71,9 @@ enum fp4_rounding {
 };
 
 /* Block Hadamard along the inner dimension [Q] "The Hadamard Transform".
- * block: 0 (none), 16, 32 or 128.  randomized: 0 = H_g, 1 = H_g diag(d)
+ * block: 0 (none), 16, 32, 64, 128 or 256 (the sizes [BG] "Block-Wise
+ * Hadamard Rotation" sweeps; 256 only for row-wise, non-transposed
+ * quantisation).  randomized: 0 = H_g, 1 = H_g diag(d)
  * with d_j = +-1 drawn from Philox(seed, counter (j/4, 0, 3, sign_tag)), one
  * pattern for every block of the tensor; two operands of one GEMM must use
  * the same seed and sign_tag so the rotations cancel [QII] MS-EDEN step 1. */
@@ -135,7 +137,8 @@ int fp4_hadamard(const void *x_dev, float *y_dev, int64_t rows, int64_t cols,
  * rotation run along x's rows -- the backward operands of [QII] "The
  * Complete Quartet II Computation Graph".  group must equal the format's
  * group size (16 NVFP4, 32 MXFP4).  cols must be a multiple of
- * max(group, had.block); with transpose = 1, in_cols must be a multiple of 8.
+ * max(group, had.block); with transpose = 1, in_cols must be a multiple of 8
+ * and had.block at most 128 (FP4_ERR_UNSUPPORTED otherwise).
  * seed/tensor_tag key the Philox streams of SR (element index in the output
  * layout) and MS-EDEN (group index).  out: caller fills the pointers; the
  * call writes rows, cols and fmt.  ws_dev: fp4_quantize_workspace_size bytes,

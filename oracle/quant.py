@@ -386,7 +386,7 @@ def supported(fmt, rnd, had_block):
     """Combinations the pages define.  Four-Over-Six and MS-EDEN are NVFP4
     methods on the Quartet II page; MS-EDEN needs a rotation (its S lives on
     rotation groups) whose blocks contain whole scale groups."""
-    if had_block not in (0, 16, 32, 128):
+    if had_block not in (0, 16, 32, 64, 128, 256):
         return False
     if fmt == MXFP4 and rnd in (FOUR_OVER_SIX, MS_EDEN):
         return False

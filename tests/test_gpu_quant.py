@@ -12,7 +12,7 @@ from oracle import quant as qn
 
 pytestmark = pytest.mark.gpu
 
-COMBOS = [(f, r, h) for f in (qn.MXFP4, qn.NVFP4) for r in range(5) for h in (0, 16, 32, 128)
+COMBOS = [(f, r, h) for f in (qn.MXFP4, qn.NVFP4) for r in range(5) for h in (0, 16, 32, 64, 128, 256)
           if qn.supported(f, r, h)]
 
 
@@ -34,6 +34,8 @@ def assert_qt_equal(g, o, check_mask=True):
 @pytest.mark.parametrize("fmt,rnd,had", COMBOS)
 @pytest.mark.parametrize("transpose", [False, True])
 def test_quantize_parity(cuda_lib, fmt, rnd, had, transpose):
+    if transpose and had > 128:
+        pytest.skip("rotation blocks above 128 are row-wise only")
     shape = (512, 200) if transpose else (200, 512)
     bits = syn.outlier_elements(shape, seed=7, stream=fmt * 10 + rnd)
     x = syn.bf16_bits_to_f32(bits)
@@ -47,6 +49,7 @@ def test_quantize_parity(cuda_lib, fmt, rnd, had, transpose):
 
 @pytest.mark.parametrize("fmt,fwd_rnd,rnd,had", [
     (qn.NVFP4, qn.FOUR_OVER_SIX, qn.MS_EDEN, 128), (qn.NVFP4, qn.FOUR_OVER_SIX, qn.SR, 16),
+    (qn.NVFP4, qn.FOUR_OVER_SIX, qn.MS_EDEN, 64),
     (qn.NVFP4, qn.RTN, qn.RTN, 0), (qn.MXFP4, qn.QUEST, qn.SR, 32), (qn.MXFP4, qn.RTN, qn.QUEST, 32)])
 @pytest.mark.parametrize("transpose", [True, False])
 def test_requantize_parity(cuda_lib, fmt, fwd_rnd, rnd, had, transpose):
@@ -66,7 +69,7 @@ def test_requantize_parity(cuda_lib, fmt, fwd_rnd, rnd, had, transpose):
     assert_qt_equal(g, o)
 
 
-@pytest.mark.parametrize("block", [16, 32, 128])
+@pytest.mark.parametrize("block", [16, 32, 64, 128, 256])
 @pytest.mark.parametrize("randomized", [False, True])
 def test_hadamard_parity(cuda_lib, block, randomized):
     bits = syn.gaussian((96, 512), 1.0, seed=5)
@@ -173,7 +176,8 @@ def test_four_over_six_grid_ties(cuda_lib, had, transpose):
     assert_qt_equal(g, o)
 
 
-@pytest.mark.parametrize("had,transpose", [(128, False), (128, True), (16, False), (32, True)])
+@pytest.mark.parametrize("had,transpose", [(128, False), (128, True), (16, False), (32, True), (64, True),
+                                          (256, False)])
 def test_ms_eden_first_pass_bit_exact(cuda_lib, had, transpose):
     """MS-EDEN's first-pass results in the workspace -- the bf16 pseudo-scales
     and the EDEN factors S = <y,y> / <y,q p> -- equal the oracle's bit for bit.
@@ -198,3 +202,10 @@ def test_ms_eden_first_pass_bit_exact(cuda_lib, had, transpose):
     np.testing.assert_array_equal(pseudo, (o.extra["pseudo"].view(np.uint32) >> 16).astype(np.uint16))
     np.testing.assert_array_equal(S, o.extra["S"].view(np.uint32))
     assert_qt_equal(g, o)
+
+
+def test_transposed_block_256_is_unsupported(cuda_lib):
+    x = to_dev(syn.gaussian((512, 256), 1.0, seed=1))
+    with pytest.raises(cuda_lib.Fp4Error) as e:
+        cuda_lib.quantize(x, qn.NVFP4, qn.RTN, 256, transpose=True)
+    assert e.value.status == 2                      # FP4_ERR_UNSUPPORTED

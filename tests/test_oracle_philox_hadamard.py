@@ -46,7 +46,7 @@ def test_philox_uniformity():
 
 
 def test_sylvester_matches_scipy_and_is_orthogonal():
-    for g in (2, 16, 32, 128):
+    for g in (2, 16, 32, 64, 128, 256):
         h = hd.sylvester(g)
         np.testing.assert_array_equal(h, scipy.linalg.hadamard(g))
         hn = h / np.sqrt(g)
@@ -55,7 +55,7 @@ def test_sylvester_matches_scipy_and_is_orthogonal():
 
 
 def test_fwht_of_basis_vectors_is_exact():
-    for g in (16, 32, 128):
+    for g in (16, 32, 64, 128, 256):
         e = np.eye(g, dtype=np.float32)
         y = hd.fwht_f32(e, g)
         want = (scipy.linalg.hadamard(g) * np.float64(hd.hadamard_scale(g))).astype(np.float32)
@@ -68,7 +68,7 @@ def test_fwht_of_basis_vectors_is_exact():
 def test_fwht_f32_close_to_exact_transform():
     rng = np.random.default_rng(0)
     x = rng.standard_normal((64, 512)).astype(np.float32)
-    for g in (16, 32, 128):
+    for g in (16, 32, 64, 128, 256):
         for rz in (False, True):
             y = hd.block_transform(x, g, rz, seed=11, sign_tag=3).astype(np.float64)
             ref = hd.block_transform_f64(x, g, rz, seed=11, sign_tag=3)
