@@ -7,9 +7,14 @@
 * Projection magnitude misalignment 1 - E[1/S], S = <X, X> / <H(X), Q(H(X))>,
   over random rotations H (Quartet page, "Backward-Pass Quantization"): zero
   for an unbiased quantiser (the page prints 0.00 for SR), non-zero for RTN.
+* Unbiasedness in the mean (Quartet II page, "Unbiasedness Verification",
+  Figure 9): the mean of B de-quantised, back-rotated samples over independent
+  rotation / rounding seeds approaches the input with an error falling like
+  1/B for an unbiased quantiser (MS-EDEN, SR), and levels off for RTN.
 
 Quantisation, rotation and de-quantisation run in the CUDA library through
-its C ABI; only the final reductions (mean square, inner products) use torch.
+its C ABI; only the final reductions (mean square, inner products) and the
+back-rotation of the de-quantised samples use torch.
 """
 import numpy as np
 import torch
@@ -66,6 +71,28 @@ def misalignment(fmt, rnd, had, rows=256, cols=4096, n_seeds=64, seed=3, device=
     return float(1.0 - v.mean()), float(v.std() / np.sqrt(v.numel()))
 
 
+def mean_convergence(fmt, rnd, had, n=10000, cols=1024, seed=14, Bs=(10, 100, 1000, 10000), device="cuda"):
+    """Relative squared error |mean_B - x|^2 / |x|^2 of the mean of the first B
+    of n samples RHT_s^-1(Q(RHT_s(x))), s = 0 .. n-1, for each B in `Bs`, and
+    the log-log slope over Bs (-1 for an unbiased quantiser).  x: 1 x cols of
+    N(0,1).  The back-rotation of seed s is the transpose of the matrix whose
+    rows are the rotated unit vectors (fp4_hadamard of the identity)."""
+    x = _dev(syn.gaussian((1, cols), 1.0, seed), device)
+    xd = x.double().view(-1)
+    eye = torch.eye(had, dtype=torch.bfloat16, device=device)
+    acc = torch.zeros((n, cols), dtype=torch.float64, device=device)
+    for s in range(n):
+        q = api.quantize(x, fmt, rnd, had, randomized=True, seed=s, sign_tag=0, tensor_tag=1)
+        dq = api.dequantize(q).double()
+        rot = api.hadamard(eye, had, randomized=True, seed=s, sign_tag=0).double()
+        acc[s] = (dq.view(-1, had) @ rot.T).view(-1)
+    Bs = [b for b in Bs if b <= n]
+    errs = [float(((acc[:b].mean(0) - xd) ** 2).sum() / (xd ** 2).sum()) for b in Bs]
+    slope = float(np.polyfit(np.log(Bs), np.log(errs), 1)[0])
+    rel_bias = float((acc.mean(0) - xd).norm() / xd.norm())
+    return {"B": Bs, "rel_sq_err": errs, "slope": slope, "rel_bias": rel_bias}
+
+
 def table(device="cuda"):
     """Every (format, rounding, rotation) the diagnostics cover, as dicts."""
     out = []
@@ -81,4 +108,7 @@ def table(device="cuda"):
         m, se = misalignment(fmt, rnd, had, device=device)
         out.append({"format": "mxfp4" if fmt == api.MXFP4 else "nvfp4", "rounding": NAMES[rnd], "had": had,
                     "misalignment": m, "misalignment_stderr": se})
+    for fmt, rnd, had in ((api.NVFP4, api.MS_EDEN, 128), (api.NVFP4, api.SR, 128), (api.NVFP4, api.RTN, 128)):
+        r = mean_convergence(fmt, rnd, had, device=device)
+        out.append({"format": "nvfp4", "rounding": NAMES[rnd], "had": had, "mean_convergence": r})
     return out

@@ -65,3 +65,17 @@ def test_misalignment_sr_zero_rtn_not(cuda_lib):
     assert abs(m_sr) < 4 * se_sr + 1e-6
     assert abs(m_eden) < 4 * se_eden + 3e-3          # MS-EDEN: unbiased to ~1e-3 (oracle pins)
     assert abs(m_rtn) > 10 * se_rtn
+
+
+def test_mean_converges_like_one_over_B(cuda_lib):
+    """Figure 9 of the Quartet II page from the CUDA path: the mean of B
+    back-rotated MS-EDEN (and SR) samples approaches the input with an error
+    falling like 1/B; RTN after a random rotation levels off."""
+    from fp4_microscaled_quantized_b200 import diagnostics as dg
+    Bs = (10, 100, 1000)
+    eden = dg.mean_convergence(qn.NVFP4, qn.MS_EDEN, 128, n=1000, Bs=Bs)
+    sr = dg.mean_convergence(qn.NVFP4, qn.SR, 128, n=1000, Bs=Bs)
+    rtn = dg.mean_convergence(qn.NVFP4, qn.RTN, 128, n=1000, Bs=Bs)
+    assert eden["slope"] <= -0.8 and sr["slope"] <= -0.8
+    assert rtn["slope"] > -0.8
+    assert eden["rel_sq_err"][-1] < rtn["rel_sq_err"][-1]
