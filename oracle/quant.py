@@ -20,7 +20,7 @@ from . import philox
 F32 = np.float32
 
 MXFP4, NVFP4 = 0, 1
-RTN, QUEST, FOUR_OVER_SIX, SR, MS_EDEN = 0, 1, 2, 3, 4
+RTN, QUEST, FOUR_OVER_SIX, SR, MS_EDEN, RTN_SQUARE16 = 0, 1, 2, 3, 4, 5
 GROUP = {MXFP4: 32, NVFP4: 16}
 
 # NVFP4 tensor-scale divisors.
@@ -123,6 +123,29 @@ def nvfp4_rtn(x, amax=None):
     d = (fm.e4m3_value(s8).astype(F32) * s32).astype(F32)
     codes, _, _ = _encode_rtn(xg, d)
     return QTensor(codes.reshape(x.shape), s8, s32, NVFP4)
+
+
+def nvfp4_rtn_square16(x, amax=None):
+    """NVFP4 round-to-nearest with one E4M3 scale per 16 x 16 block (the
+    square-block weight quantisation of the NVIDIA recipe, Quartet II page,
+    "The square-block trade-off" and Table 1 "16x16"): the block maximum takes
+    the place of the 1 x 16 group maximum in the RTN rule.  The scales are
+    returned per 1 x 16 group (rows x cols/16, each block's scale repeated on
+    its 16 rows), the layout the block-scaled GEMM reads.  Rows and columns
+    are multiples of 16.  Quantising x^T gives the transpose of quantising x
+    (the blocks and the rule are symmetric), which is what lets the recipe
+    re-use Q(W) for W^T."""
+    x = np.asarray(x, dtype=F32)
+    rows, cols = x.shape
+    assert rows % 16 == 0 and cols % 16 == 0, "16 x 16 blocks need rows and cols divisible by 16"
+    amax = abs_max(x) if amax is None else F32(amax)
+    s32 = nvfp4_tensor_scale(amax, NV_RTN_DIV)
+    bmax = np.abs(x).reshape(rows // 16, 16, cols // 16, 16).max(axis=(1, 3)).astype(F32)
+    sb = fm.rtn_e4m3((bmax / F32(s32 * F32(6.0))).astype(F32))
+    s8 = np.repeat(sb, 16, axis=0)                       # rows x cols/16
+    d = (fm.e4m3_value(s8).astype(F32) * s32).astype(F32)
+    codes, _, _ = _encode_rtn(_groups(x, 16), d)
+    return QTensor(codes.reshape(x.shape), s8.astype(np.uint8), s32, NVFP4)
 
 
 def nvfp4_four_over_six(x, amax=None):
@@ -392,6 +415,8 @@ def supported(fmt, rnd, had_block):
         return False
     if rnd == MS_EDEN and (had_block == 0 or had_block < GROUP[fmt]):
         return False
+    if rnd == RTN_SQUARE16 and (fmt != NVFP4 or had_block != 0):
+        return False
     return True
 
 
@@ -411,6 +436,8 @@ def quantize_transformed(y, fmt, rnd, seed=0, tensor_tag=0, chunk=None, amax=Non
             return nvfp4_quest(y, amax)
         if rnd == MS_EDEN:
             return nvfp4_ms_eden(y, chunk, seed, tensor_tag, amax, row_ids)
+        if rnd == RTN_SQUARE16:
+            return nvfp4_rtn_square16(y, amax)
     else:
         if rnd == RTN:
             return mxfp4_rtn(y)

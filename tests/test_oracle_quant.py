@@ -331,3 +331,43 @@ def test_ms_eden_unbiased_and_1_over_B():
     err = [np.sum((acc[:b].mean(0) - x[0]) ** 2) / np.sum(x[0].astype(np.float64) ** 2) for b in Bs]
     slope = np.polyfit(np.log(Bs), np.log(err), 1)[0]
     assert slope <= -0.8
+
+
+# ------------------------------------------- 16 x 16 square-block scales ----
+def test_table1_square_block_rtn(gauss_1m):
+    """Quartet II page, Table 1: RTN with 16 x 16 scales, MSE 12.4e-3 (worse
+    than native 1 x 16 RTN)."""
+    m = _mse(qn.nvfp4_rtn_square16(gauss_1m), gauss_1m)
+    assert m == pytest.approx(T1["mse_x1e3"]["RTN 16x16"], rel=0.03)
+    assert m > _mse(qn.nvfp4_rtn(gauss_1m), gauss_1m)
+
+
+def test_square_block_scales_and_codes_from_the_definition():
+    """Every element against the rule written out in fp64 decisions: the
+    block's scale is RTN_E4M3(block max / (s32 * 6)), shared by the block's 16
+    rows, the code is RTN_E2M1 of x / (scale * s32)."""
+    x = _gauss((32, 48), 21) * F32(3.0)
+    q = qn.nvfp4_rtn_square16(x)
+    amax = np.max(np.abs(x))
+    s32 = F32(F32(amax) / F32(1536.0))
+    for br in range(2):
+        for bc in range(3):
+            blk = x[16 * br:16 * br + 16, 16 * bc:16 * bc + 16]
+            s8 = int(fm.rtn_e4m3(np.array([F32(np.max(np.abs(blk))) / F32(s32 * F32(6.0))], F32))[0])
+            assert np.all(q.scales[16 * br:16 * br + 16, bc] == s8)
+            d = F32(F32(fm.e4m3_value(np.array([s8]))[0]) * s32)
+            inv = F32(F32(1.0) / d)
+            v = (blk * inv).astype(F32)
+            want = fm.rtn_e2m1(v)
+            np.testing.assert_array_equal(q.codes[16 * br:16 * br + 16, 16 * bc:16 * bc + 16], want)
+
+
+def test_square_block_quantisation_commutes_with_transpose():
+    """Q(x^T) = Q(x)^T for 16 x 16 blocks: the NVIDIA recipe's re-use of the
+    forward Q(W) as Q(W^T) in the dX GEMM (Quartet II page)."""
+    x = _gauss((64, 96), 22)
+    a = qn.nvfp4_rtn_square16(x)
+    b = qn.quantize(x, qn.NVFP4, qn.RTN_SQUARE16, 0, transpose=True)
+    np.testing.assert_array_equal(b.codes, a.codes.T)
+    np.testing.assert_array_equal(b.scales, np.repeat(a.scales[::16].T, 16, axis=0))
+    assert b.tensor_scale == a.tensor_scale
