@@ -342,13 +342,14 @@ def run_e2e(api, M, steps, device, host):
 
 # ------------------------------------------------------ quantiser sweep --
 SWEEP_COLS = 4096
-RND_NAMES = {0: "rtn", 1: "quest", 2: "fos", 3: "sr", 4: "eden"}
+RND_NAMES = {0: "rtn", 1: "quest", 2: "fos", 3: "sr", 4: "eden", 5: "rtn16x16"}
 
 
 def sweep_cases(api):
     """(name, fmt, rounding, had_block, randomized) of every combination the C ABI
     accepts: MXFP4 (RTN, QuEST, SR) and NVFP4 (RTN, QuEST, 4/6, SR) with Hadamard
-    none/16/32/64/128/256, NVFP4 MS-EDEN with 16/32/64/128/256.  The stochastic modes use the
+    none/16/32/64/128/256, NVFP4 MS-EDEN with 16/32/64/128/256, NVFP4 RTN with
+    16 x 16 block scales.  The stochastic modes use the
     randomized transform (backward pass), the others the deterministic one."""
     out = []
     for fmt, fname, rnds in ((api.MXFP4, "mxfp4", (api.RTN, api.QUEST, api.SR)),
@@ -360,13 +361,14 @@ def sweep_cases(api):
                     continue
                 rand = rnd in (api.SR, api.MS_EDEN) and had > 0
                 out.append(("%s-%s-h%d" % (fname, RND_NAMES[rnd], had), fmt, rnd, had, rand))
+    out.append(("nvfp4-rtn16x16-h0", api.NVFP4, api.RTN_SQUARE16, 0, False))
     return out
 
 
 def sweep_bytes_per_elem(api, fmt, rnd, had):
     """Algorithmic HBM bytes per element of one quantise call: bf16 read 2 B,
     codes 0.5, one scale copy 1/g; NVFP4 global-scale modes read the input
-    twice (amax pass); QuEST writes a 1-bit mask; MS-EDEN writes and re-reads
+    twice (amax or 16 x 16 block-maximum pass); QuEST writes a 1-bit mask; MS-EDEN writes and re-reads
     bf16 pseudo-scales (2 x 2/16) and fp32 EDEN factors (2 x 4/had)."""
     g = api.GROUP[fmt]
     b = 2.0 + 0.5 + 1.0 / g

@@ -15,7 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfp4_b200.so")
 
 MXFP4, NVFP4 = 0, 1
-RTN, QUEST, FOUR_OVER_SIX, SR, MS_EDEN = 0, 1, 2, 3, 4
+RTN, QUEST, FOUR_OVER_SIX, SR, MS_EDEN, RTN_SQUARE16 = 0, 1, 2, 3, 4, 5
 GROUP = {MXFP4: 32, NVFP4: 16}
 
 STATUS = {0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED", 3: "FP4_ERR_ALIGNMENT",

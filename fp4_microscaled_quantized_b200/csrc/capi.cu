@@ -45,12 +45,15 @@ static inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<u
 static inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
 struct WsLayout {
-  size_t amax = 0, pseudo = 0, eden = 0, total = 0;
+  size_t amax = 0, pseudo = 0, eden = 0, bmax = 0, total = 0;
 };
 
 static WsLayout ws_layout(int64_t rows, int64_t cols, int fmt, int rnd, int had) {
   WsLayout w;
-  if (fmt == FP4_NVFP4 && rnd == FP4_MS_EDEN && had > 0) {
+  if (fmt == FP4_NVFP4 && rnd == FP4_RTN_SQUARE16) {
+    w.bmax = 256;
+    w.total = w.bmax + align256(size_t(rows / 16) * size_t(cols / 16) * 4);
+  } else if (fmt == FP4_NVFP4 && rnd == FP4_MS_EDEN && had > 0) {
     w.amax = 0;
     w.pseudo = 256;
     w.eden = w.pseudo + align256(size_t(rows) * size_t(cols / 16) * 2);
@@ -66,6 +69,7 @@ static bool combo_supported(int fmt, int rnd, int had) {
   if (fmt == FP4_MXFP4 && (rnd == FP4_FOUR_OVER_SIX || rnd == FP4_MS_EDEN)) return false;
   int g = fmt == FP4_NVFP4 ? 16 : 32;
   if (rnd == FP4_MS_EDEN && (had == 0 || had < g)) return false;
+  if (rnd == FP4_RTN_SQUARE16 && (fmt != FP4_NVFP4 || had != 0)) return false;
   return true;
 }
 
@@ -130,6 +134,37 @@ static int launch_pad(uint8_t* swz, int64_t rows, int64_t ng, cudaStream_t s) {
 }
 
 // Shared sequencing of fp4_quantize / fp4_requantize.
+// Maxima |x| of the 16 x 16 blocks of a bf16 tensor (rows x cols, both
+// multiples of 16), one block per thread (consecutive threads: consecutive
+// blocks of a block row, so each of the 16 row loads of a warp is one
+// contiguous run), as fp32 bits; the block-wide maximum goes to the global
+// amax word.  With the sign bit cleared, |x| orders as an unsigned 16-bit
+// integer (NaN patterns above infinity).
+__global__ void __launch_bounds__(256) k_block16_max(const uint16_t* x, int64_t rows, int64_t cols, uint32_t* bmax,
+                                                     uint32_t* amax, int* status) {
+  __shared__ Shared sh;
+  const int64_t nbc = cols >> 4, nb = (rows >> 4) * nbc;
+  uint32_t acc = 0;
+  for (int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; b < nb; b += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t br = b / nbc, bc = b - br * nbc;
+    const uint16_t* src = x + (br << 4) * cols + (bc << 4);
+    uint32_t m2 = 0;
+#pragma unroll 4
+    for (int r = 0; r < 16; ++r) {
+      const uint4* row = reinterpret_cast<const uint4*>(src + r * cols);
+      const uint4 u = __ldg(row), v = __ldg(row + 1);
+      m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu),
+                                 __vmaxu2(u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu)));
+      m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                 __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+    }
+    const uint32_t m = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+    bmax[b] = m;
+    acc = max(acc, m);
+  }
+  block_max_atomic(acc, sh, amax, status);
+}
+
 static int run_quant(int load, int fmt, int rnd, int had, QParams& p, void* ws, size_t ws_bytes,
                      cudaStream_t s) {
   WsLayout L = ws_layout(p.rows, p.cols, fmt, rnd, had);
@@ -141,6 +176,7 @@ static int run_quant(int load, int fmt, int rnd, int had, QParams& p, void* ws, 
   p.amax_bits = L.total ? reinterpret_cast<uint32_t*>(w + L.amax) : nullptr;
   p.pseudo = (L.pseudo ? reinterpret_cast<uint16_t*>(w + L.pseudo) : nullptr);
   p.eden_S = (L.eden ? reinterpret_cast<float*>(w + L.eden) : nullptr);
+  uint32_t* bmax = L.bmax ? reinterpret_cast<uint32_t*>(w + L.bmax) : nullptr;
   p.status = status_ptr();
   p.nkb = ((p.cols / (fmt == FP4_NVFP4 ? 16 : 32)) + 3) / 4;
   auto launch = [&](int r) -> cudaError_t {
@@ -153,9 +189,24 @@ static int run_quant(int load, int fmt, int rnd, int had, QParams& p, void* ws, 
   };
   if (fmt == FP4_NVFP4) {
     if (cudaMemsetAsync(p.amax_bits, 0, sizeof(uint32_t), s) != cudaSuccess) return FP4_ERR_CUDA;
-    if (rnd != FP4_MS_EDEN && launch(R_AMAX) != cudaSuccess) return FP4_ERR_CUDA;
+    if (rnd == FP4_RTN_SQUARE16) {
+      // block maxima of the input (and the global amax with them)
+      const int64_t nb = (p.in_rows / 16) * (p.in_cols / 16);
+      int64_t blocks = (nb + 255) / 256, cap = int64_t(num_sms()) * 8;
+      if (blocks > cap) blocks = cap;
+      if (blocks < 1) blocks = 1;
+      k_block16_max<<<unsigned(blocks), 256, 0, s>>>(static_cast<const uint16_t*>(p.x), p.in_rows, p.in_cols,
+                                                     bmax, p.amax_bits, p.status);
+      count_launch();
+      if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
+      p.bmax = bmax;
+      p.bmax_ld = p.in_cols / 16;
+      p.bmax_trans = load == LD_TRANS ? 1 : 0;
+    } else if (rnd != FP4_MS_EDEN && launch(R_AMAX) != cudaSuccess) {
+      return FP4_ERR_CUDA;
+    }
   }
-  if (launch(rnd) != cudaSuccess) return FP4_ERR_CUDA;
+  if (launch(rnd == FP4_RTN_SQUARE16 ? R_SQ16 : rnd) != cudaSuccess) return FP4_ERR_CUDA;
   if (rnd == FP4_MS_EDEN) {
     int64_t groups = p.rows * (p.cols / 16);
     int64_t blocks = (groups + 255) / 256, cap = int64_t(num_sms()) * 8;
@@ -194,10 +245,13 @@ int fp4_quantize(const void* x, int64_t in_rows, int64_t in_cols, int32_t transp
                  int32_t rounding, int32_t group, fp4_had had, uint64_t seed, uint32_t tensor_tag,
                  fp4_qtensor* out, void* ws, size_t ws_bytes, fp4_stream_t stream) {
   if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
-  if (rounding < FP4_RTN || rounding > FP4_MS_EDEN) return FP4_ERR_INVALID_ARG;
+  if (rounding < FP4_RTN || rounding > FP4_RTN_SQUARE16) return FP4_ERR_INVALID_ARG;
   const int g = fmt == FP4_NVFP4 ? 16 : 32;
   if (group != g) return FP4_ERR_UNSUPPORTED;
   if (!combo_supported(fmt, rounding, had.block)) return FP4_ERR_UNSUPPORTED;
+  // square blocks: whole 16 x 16 blocks and 32-element rows of the output
+  if (rounding == FP4_RTN_SQUARE16 && (in_rows % 16 || in_cols % 16 || (transpose ? in_rows : in_cols) % 32))
+    return FP4_ERR_INVALID_ARG;
   if (in_rows < 0 || in_cols < 0 || (transpose != 0 && transpose != 1) || !out)
     return FP4_ERR_INVALID_ARG;
   const int64_t rows = transpose ? in_cols : in_rows, cols = transpose ? in_rows : in_cols;
@@ -227,8 +281,9 @@ int fp4_requantize(const fp4_qtensor* in, int32_t transpose, int32_t rounding, f
   if ((in->rows > 0 && in->cols > 0) && (!in->codes || !in->scales || !in->tensor_scale))
     return FP4_ERR_INVALID_ARG;
   if (in->fmt != FP4_MXFP4 && in->fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
-  if (rounding < FP4_RTN || rounding > FP4_MS_EDEN || (transpose != 0 && transpose != 1))
+  if (rounding < FP4_RTN || rounding > FP4_RTN_SQUARE16 || (transpose != 0 && transpose != 1))
     return FP4_ERR_INVALID_ARG;
+  if (rounding == FP4_RTN_SQUARE16) return FP4_ERR_UNSUPPORTED;   // bf16 input only
   const int fmt = in->fmt, g = fmt == FP4_NVFP4 ? 16 : 32;
   if (!combo_supported(fmt, rounding, had.block)) return FP4_ERR_UNSUPPORTED;
   if (in->rows < 0 || in->cols < 0 || in->cols % g || !out) return FP4_ERR_INVALID_ARG;

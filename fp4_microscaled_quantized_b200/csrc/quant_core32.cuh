@@ -269,14 +269,22 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
   uint32_t sb[NG];
   uint32_t mbits = 0;
 
-  if (FMT == FMT_NV && (RND == R_RTN || RND == R_FOS || RND == R_SR || RND == R_QUEST)) {
+  if (FMT == FMT_NV && (RND == R_RTN || RND == R_SQ16 || RND == R_FOS || RND == R_SR || RND == R_QUEST)) {
     const float s32 = qc.s32;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       const float* xg = x + 16 * g;
       const float gmax = bitsf(gmb[g]);
       uint32_t* wg = w + 2 * g;
-      if (RND == R_RTN) {
+      if (RND == R_SQ16) {
+        // RTN against the maximum of the group's 16 x 16 block of the input
+        const int64_t oc = (ocol >> 4) + g, orb = orow >> 4;
+        const float bm = bitsf(p.bmax[p.bmax_trans ? oc * p.bmax_ld + orb : orb * p.bmax_ld + oc]);
+        const uint32_t s8 = e4m3_rtn(exact_div(bm, qc.d6));
+        const float d = __fmul_rn(e4m3x2_value(s8).x, s32), inv = __frcp_rn(d);
+        enc16(xg, inv, finite_pos(d, inv), wg);
+        sb[g] = s8;
+      } else if (RND == R_RTN) {
         const uint32_t s8 = e4m3_rtn(exact_div(gmax, qc.d6));
         const float d = __fmul_rn(e4m3x2_value(s8).x, s32), inv = __frcp_rn(d);
         enc16(xg, inv, finite_pos(d, inv), wg);
@@ -487,7 +495,7 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
 // SR and QuEST keep their registers.
 template <int RND>
 __host__ __device__ constexpr int quant_min_blocks() {
-  return (RND == R_RTN || RND == R_AMAX) ? 4 : ((RND == R_FOS || RND == R_EDEN) ? 3 : 1);
+  return (RND == R_RTN || RND == R_SQ16 || RND == R_AMAX) ? 4 : ((RND == R_FOS || RND == R_EDEN) ? 3 : 1);
 }
 // The transposed kernel's shared-memory tile allows 6 blocks per SM; its
 // compute phase needs fewer registers, and 4 resident blocks overlap one

@@ -32,8 +32,9 @@ int resident_blocks() {
 template <int LOAD, int FMT, int RND, int HAD>
 cudaError_t launch_one(const QParams& p, cudaStream_t s) {
   constexpr bool TRANS = LOAD == LD_TRANS || LOAD == LD_TRANS_FP4;
-  if constexpr (TRANS && HAD > 128) {
-    // a rotation block longer than the transposed kernel's 128-row tile
+  if constexpr ((TRANS && HAD > 128) || (RND == R_SQ16 && (HAD != 0 || LOAD == LD_ROW_FP4 || LOAD == LD_TRANS_FP4))) {
+    // a rotation block longer than the transposed kernel's 128-row tile;
+    // square blocks: bf16 input, no rotation
     return cudaErrorInvalidValue;
   } else {
     const bool wide = (p.cols % 32) == 0;   // 32 elements per lane (always so for blocks >= 32)
@@ -50,7 +51,7 @@ cudaError_t launch_one(const QParams& p, cudaStream_t s) {
                 unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
       k_quant_trans32<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
       count_launch();
-    } else if constexpr (HAD <= 16) {
+    } else if constexpr (HAD <= 16 && RND != R_SQ16) {
       // inner dimension 16 mod 32: 8 elements per lane
       if (!TRANS) {
         int64_t tasks = p.rows * (p.cols >> 3);
@@ -106,6 +107,7 @@ cudaError_t launch_one(const QParams& p, cudaStream_t s) {
         case R_FOS: { FP4_HAD_SWITCH(LOAD, FMT_NV, R_FOS) }                         \
         case R_SR: { FP4_HAD_SWITCH(LOAD, FMT_NV, R_SR) }                           \
         case R_EDEN: { FP4_HAD_SWITCH_ROT(LOAD, FMT_NV, R_EDEN) }                   \
+        case R_SQ16: return launch_one<LOAD, FMT_NV, R_SQ16, 0>(p, s);              \
         default: return cudaErrorInvalidValue;                                      \
       }                                                                             \
     }                                                                               \

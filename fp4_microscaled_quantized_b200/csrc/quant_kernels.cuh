@@ -15,7 +15,8 @@
 namespace fp4 {
 
 enum : int { FMT_MX = 0, FMT_NV = 1 };
-enum : int { R_RTN = 0, R_QUEST = 1, R_FOS = 2, R_SR = 3, R_EDEN = 4, R_AMAX = 5 };
+// R_AMAX: the global amax pass; R_SQ16: RTN against 16 x 16 block maxima.
+enum : int { R_RTN = 0, R_QUEST = 1, R_FOS = 2, R_SR = 3, R_EDEN = 4, R_AMAX = 5, R_SQ16 = 6 };
 enum : int { LD_ROW = 0, LD_TRANS = 1, LD_ROW_FP4 = 2, LD_TRANS_FP4 = 3 };
 
 struct QParams {
@@ -38,6 +39,11 @@ struct QParams {
   uint32_t tensor_tag;
   uint32_t sign_tag;
   int32_t randomized;
+  // 16 x 16 block maxima (fp32 bits) of the input, row-major with ld
+  // columns; trans: the quantised tensor is the input's transpose
+  const uint32_t* bmax;
+  int64_t bmax_ld;
+  int32_t bmax_trans;
   // workspace
   uint32_t* amax_bits;
   uint16_t* pseudo;

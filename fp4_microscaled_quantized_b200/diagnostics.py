@@ -2,7 +2,8 @@
 
 * Quantisation MSE on N(0, 1) vectors for every format and rounding mode --
   the Quartet II page's Table 1 ("Practical Performance of MS-EDEN": NVFP4
-  SR 23.5, MS-EDEN 9.8, RTN 9.0, RTN + 4/6 7.6, all x 1e-3) and the MXFP4
+  SR 23.5, MS-EDEN 9.8, RTN 9.0, RTN + 4/6 7.6, RTN with 16 x 16 scales 12.4,
+  all x 1e-3) and the MXFP4
   error column of the Quartet page's Table 2.
 * Projection magnitude misalignment 1 - E[1/S], S = <X, X> / <H(X), Q(H(X))>,
   over random rotations H (Quartet page, "Backward-Pass Quantization"): zero
@@ -23,9 +24,10 @@ from . import api
 from . import synthetic as syn
 
 # Table 1 of the Quartet II page (NVFP4, native 1x16 scales, MSE x 1e-3).
-TABLE1_NVFP4 = {"rtn": 9.0, "fos": 7.6, "sr": 23.5, "eden": 9.8}
+TABLE1_NVFP4 = {"rtn": 9.0, "fos": 7.6, "sr": 23.5, "eden": 9.8, "rtn16x16": 12.4}
 
-NAMES = {api.RTN: "rtn", api.QUEST: "quest", api.FOUR_OVER_SIX: "fos", api.SR: "sr", api.MS_EDEN: "eden"}
+NAMES = {api.RTN: "rtn", api.QUEST: "quest", api.FOUR_OVER_SIX: "fos", api.SR: "sr", api.MS_EDEN: "eden",
+         api.RTN_SQUARE16: "rtn16x16"}
 
 
 def _dev(bits, device):
@@ -96,7 +98,7 @@ def mean_convergence(fmt, rnd, had, n=10000, cols=1024, seed=14, Bs=(10, 100, 10
 def table(device="cuda"):
     """Every (format, rounding, rotation) the diagnostics cover, as dicts."""
     out = []
-    for rnd, had in ((api.RTN, 0), (api.FOUR_OVER_SIX, 0), (api.SR, 0), (api.MS_EDEN, 128)):
+    for rnd, had in ((api.RTN, 0), (api.FOUR_OVER_SIX, 0), (api.SR, 0), (api.MS_EDEN, 128), (api.RTN_SQUARE16, 0)):
         out.append({"format": "nvfp4", "rounding": NAMES[rnd], "had": had,
                     "mse_x1e3": quant_mse(api.NVFP4, rnd, had, device=device),
                     "page_mse_x1e3": TABLE1_NVFP4[NAMES[rnd]]})

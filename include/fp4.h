@@ -67,7 +67,13 @@ enum fp4_rounding {
   FP4_QUEST = 1,         /* RMSE-optimal clipping + clip mask [Q] "QuEST in Detail" */
   FP4_FOUR_OVER_SIX = 2, /* NVFP4 only [QII] "Forward Pass Design"                  */
   FP4_SR = 3,            /* NVFP4: [QII] standard SR steps 1-3; MXFP4: SR(3/4 x) [Q] */
-  FP4_MS_EDEN = 4        /* NVFP4 only, needs a rotation [QII] MS-EDEN, post hoc     */
+  FP4_MS_EDEN = 4,       /* NVFP4 only, needs a rotation [QII] MS-EDEN, post hoc     */
+  FP4_RTN_SQUARE16 = 5   /* NVFP4 RTN, one scale per 16 x 16 block [QII] "The
+                            square-block trade-off"; no rotation, rows a multiple
+                            of 16, cols of 32; bf16 input only (not for
+                            fp4_requantize); scales stored per 1 x 16 group, each
+                            block's scale repeated on its 16 rows.  Quantising
+                            x^T gives the transpose of quantising x.            */
 };
 
 /* Block Hadamard along the inner dimension [Q] "The Hadamard Transform".
@@ -101,7 +107,9 @@ typedef struct {
  * quantised tensor of rows x cols (16-byte multiple; 0 for modes without a
  * global pass).  NVFP4 RTN/QuEST/4-6/SR: one amax word.  MS-EDEN: amax, the
  * bf16 E8M3 pseudo-scales (rows * cols/16 * 2) and the fp32 EDEN factors
- * (rows * cols/block * 4) of the post hoc range alignment [QII].  Layout:
+ * (rows * cols/block * 4) of the post hoc range alignment [QII].  Square
+ * blocks: amax and the fp32 maxima of the 16 x 16 blocks (rows/16 * cols/16
+ * * 4 at byte 256).  MS-EDEN layout:
  * the amax bits (uint32) at byte 0; the pseudo-scales, row-major, at byte
  * 256; the EDEN factors, row-major, at byte 256 + the pseudo-scale bytes
  * rounded up to a multiple of 256.  After an MS-EDEN call the workspace

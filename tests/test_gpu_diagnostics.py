@@ -46,7 +46,8 @@ def test_table1_from_gpu_quantisers(cuda_lib):
     bits = syn.gaussian((1024, 1024), 1.0, 0)
     x = syn.bf16_bits_to_f32(bits)
     for rnd, had, page, rel in ((qn.RTN, 0, 9.0, 0.03), (qn.FOUR_OVER_SIX, 0, 7.6, 0.03),
-                                (qn.SR, 0, 23.5, 0.03), (qn.MS_EDEN, 128, 9.8, 0.05)):
+                                (qn.SR, 0, 23.5, 0.03), (qn.MS_EDEN, 128, 9.8, 0.05),
+                                (qn.RTN_SQUARE16, 0, 12.4, 0.03)):
         gpu = dg.quant_mse(qn.NVFP4, rnd, had, n_seeds=1)
         assert gpu == pytest.approx(page, rel=rel)
         # the same value from the oracle's quantisation of the same input

@@ -209,3 +209,46 @@ def test_transposed_block_256_is_unsupported(cuda_lib):
     with pytest.raises(cuda_lib.Fp4Error) as e:
         cuda_lib.quantize(x, qn.NVFP4, qn.RTN, 256, transpose=True)
     assert e.value.status == 2                      # FP4_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("transpose", [False, True])
+@pytest.mark.parametrize("shape", [(64, 512), (320, 1024), (1024, 96)])
+def test_square_block_parity(cuda_lib, shape, transpose):
+    """NVFP4 RTN with 16 x 16 block scales: codes, scales (repeated on each
+    block's rows) and tensor scale bit-exact against the oracle."""
+    in_shape = (shape[1], shape[0]) if transpose else shape
+    if (in_shape[0] if transpose else in_shape[1]) % 32:
+        pytest.skip("square blocks need 32-element output rows")
+    bits = syn.outlier_elements(in_shape, seed=13, stream=shape[0])
+    x = syn.bf16_bits_to_f32(bits)
+    g = cuda_lib.quantize(to_dev(bits), qn.NVFP4, qn.RTN_SQUARE16, 0, transpose=transpose)
+    o = qn.quantize(x, qn.NVFP4, qn.RTN_SQUARE16, 0, transpose=transpose)
+    assert_qt_equal(g, o)
+    assert cuda_lib.get_last_error() == 0
+
+
+def test_square_block_transpose_is_the_transpose(cuda_lib):
+    """Quantising W^T with 16 x 16 blocks gives the transpose of Q(W) -- the
+    property that lets the NVIDIA recipe re-use the forward Q(W) for W^T."""
+    bits = syn.gaussian((256, 512), 0.02, seed=4)
+    d = to_dev(bits)
+    a = cuda_lib.quantize(d, qn.NVFP4, qn.RTN_SQUARE16, 0)
+    b = cuda_lib.quantize(d, qn.NVFP4, qn.RTN_SQUARE16, 0, transpose=True)
+    torch.cuda.synchronize()
+    ca = fm.unpack_codes(a.codes.cpu().numpy())
+    cb = fm.unpack_codes(b.codes.cpu().numpy())
+    np.testing.assert_array_equal(cb, ca.T)
+    sa, sbt = a.scales.cpu().numpy(), b.scales.cpu().numpy()
+    np.testing.assert_array_equal(sbt, np.repeat(sa[::16].T, 16, axis=0))
+
+
+def test_square_block_argument_errors(cuda_lib):
+    x = to_dev(syn.gaussian((72, 256), 1.0, seed=1))          # 72 rows: not whole blocks
+    with pytest.raises(cuda_lib.Fp4Error) as e:
+        cuda_lib.quantize(x, qn.NVFP4, qn.RTN_SQUARE16, 0)
+    assert e.value.status == 1
+    y = to_dev(syn.gaussian((64, 256), 1.0, seed=1))
+    for fmt, had in ((qn.MXFP4, 0), (qn.NVFP4, 16)):
+        with pytest.raises(cuda_lib.Fp4Error) as e:
+            cuda_lib.quantize(y, fmt, qn.RTN_SQUARE16, had)
+        assert e.value.status == 2

@@ -252,7 +252,11 @@ def test_unsupported_combinations():
     assert not qn.supported(qn.MXFP4, qn.MS_EDEN, 128)
     assert not qn.supported(qn.NVFP4, qn.MS_EDEN, 0)
     assert qn.supported(qn.NVFP4, qn.MS_EDEN, 16)
-    assert not qn.supported(qn.NVFP4, qn.RTN, 64)
+    assert qn.supported(qn.NVFP4, qn.RTN, 64) and qn.supported(qn.NVFP4, qn.MS_EDEN, 256)
+    assert not qn.supported(qn.NVFP4, qn.RTN, 8) and not qn.supported(qn.NVFP4, qn.RTN, 512)
+    assert qn.supported(qn.NVFP4, qn.RTN_SQUARE16, 0)
+    assert not qn.supported(qn.MXFP4, qn.RTN_SQUARE16, 0)
+    assert not qn.supported(qn.NVFP4, qn.RTN_SQUARE16, 16)
     with pytest.raises(ValueError):
         qn.quantize(np.zeros((1, 32), F32), qn.MXFP4, qn.MS_EDEN, 128, True)
 
