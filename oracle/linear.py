@@ -12,6 +12,16 @@ Test infrastructure only (see ``oracle/__init__.py``).
   transpose, RHT128 on the inner dimension and MS-EDEN for (E, W^T) and
   (E^T, X^T); no inverse transform.
 * RTN -- a single NVFP4 RTN linear layer without rotation.
+* NVIDIA -- the NVIDIA recipe the Quartet II page describes ("The
+  square-block trade-off"; "Comparison to TetraJet-v2 and the NVIDIA
+  recipe"): forward X with native 1x16 RTN scales, W with 16x16 square-block
+  RTN scales, no rotation; backward SR; the dX GEMM re-uses the forward Q(W),
+  transposed, with dY quantised along N without a rotation (the rotation must
+  act on both operands of a GEMM, and W is re-used as it is); the dW GEMM
+  rotates both operands (SR of RHT(dY^T) and of RHT(Q(X)^T)).  READINGS: the
+  page does not give the dW GEMM's operands beyond "RHT only on the backward
+  pass"; X^T is re-quantised from the saved Q(X) as in the other recipes, and
+  the rotation block is 16, the square block size.
 * TETRAJET2 -- the simplified TetraJet-v2 of the Quartet II page ("Comparison
   to TetraJet-v2 and the NVIDIA recipe"): NVFP4 RTN with native 1x16 scales
   on the forward pass, SR with the RHT on the inner dimension for both
@@ -45,18 +55,22 @@ class Recipe:
     bwd_had: int
     bwd_randomized: bool
     mask_epilogue: bool
+    w_rnd: int = -1          # forward rounding of W (-1: fwd_rnd)
+    w_reuse: bool = False    # dX GEMM re-uses Q(W)^T; dY quantised without rotation
 
 
 QUARTET = Recipe(qn.MXFP4, qn.QUEST, 32, qn.SR, 32, True, True)
 QUARTET2 = Recipe(qn.NVFP4, qn.FOUR_OVER_SIX, 0, qn.MS_EDEN, 128, True, False)
 RTN = Recipe(qn.NVFP4, qn.RTN, 0, qn.RTN, 0, False, False)
 TETRAJET2 = Recipe(qn.NVFP4, qn.RTN, 0, qn.SR, 128, True, False)
+NVIDIA = Recipe(qn.NVFP4, qn.RTN, 0, qn.SR, 16, True, False, w_rnd=qn.RTN_SQUARE16, w_reuse=True)
 
 
 def linear_fwd(X, W, r, seed=0):
     """Returns (Y_ref, bound, ctx) with ctx = {"Xq", "Wq"}."""
     Xq = qn.quantize(X, r.fmt, r.fwd_rnd, r.fwd_had, False, seed, 0, TAG_X)
-    Wq = qn.quantize(W, r.fmt, r.fwd_rnd, r.fwd_had, False, seed, 0, TAG_W)
+    w_rnd = r.fwd_rnd if r.w_rnd < 0 else r.w_rnd
+    Wq = qn.quantize(W, r.fmt, w_rnd, r.fwd_had, False, seed, 0, TAG_W)
     y, b = gm.gemm_ref(Xq, Wq)
     return y, b, {"Xq": Xq, "Wq": Wq}
 
@@ -64,8 +78,12 @@ def linear_fwd(X, W, r, seed=0):
 def bwd_operands(dY, ctx, r, step_seed):
     """The four backward operands, quantised along each GEMM's inner dim."""
     h, rz, s = r.bwd_had, r.bwd_randomized, step_seed
-    E_row = qn.quantize(dY, r.fmt, r.bwd_rnd, h, rz, s, GEMM_DX, TAG_E_ROW)
-    W_t = qn.requantize(ctx["Wq"], r.bwd_rnd, h, rz, s, GEMM_DX, TAG_W_T, transpose=True)
+    if r.w_reuse:
+        E_row = qn.quantize(dY, r.fmt, r.bwd_rnd, 0, False, s, GEMM_DX, TAG_E_ROW)
+        W_t = qn.transpose_square16(ctx["Wq"])
+    else:
+        E_row = qn.quantize(dY, r.fmt, r.bwd_rnd, h, rz, s, GEMM_DX, TAG_E_ROW)
+        W_t = qn.requantize(ctx["Wq"], r.bwd_rnd, h, rz, s, GEMM_DX, TAG_W_T, transpose=True)
     E_t = qn.quantize(dY, r.fmt, r.bwd_rnd, h, rz, s, GEMM_DW, TAG_E_T, transpose=True)
     X_t = qn.requantize(ctx["Xq"], r.bwd_rnd, h, rz, s, GEMM_DW, TAG_X_T, transpose=True)
     return {"E_row": E_row, "W_t": W_t, "E_t": E_t, "X_t": X_t}

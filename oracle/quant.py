@@ -148,6 +148,17 @@ def nvfp4_rtn_square16(x, amax=None):
     return QTensor(codes.reshape(x.shape), s8.astype(np.uint8), s32, NVFP4)
 
 
+def transpose_square16(qt):
+    """The transpose of a 16 x 16 square-block quantised tensor: codes
+    transposed, each block's scale moved to the transposed block (the
+    re-use of Q(W) as Q(W^T) in the NVIDIA recipe's dX GEMM)."""
+    rows, cols = qt.codes.shape
+    assert qt.fmt == NVFP4 and rows % 16 == 0 and cols % 16 == 0
+    sb = qt.scales[::16]                                  # block scales (rows/16 x cols/16)
+    return QTensor(np.ascontiguousarray(qt.codes.T), np.repeat(sb.T, 16, axis=0).astype(np.uint8),
+                   qt.tensor_scale, NVFP4)
+
+
 def nvfp4_four_over_six(x, amax=None):
     """Four-Over-Six (Quartet II page, "Forward Pass Design", steps 1-4): per
     block of 16, quantise once with the block maximum mapped to 6 and once

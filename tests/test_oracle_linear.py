@@ -71,7 +71,7 @@ def test_quartet_forward_and_backward_track_exact_gradients():
     assert float(ops["E_row"].tensor_scale) * float(ops["W_t"].tensor_scale) == np.float32(4 / 3) ** 2
 
 
-@pytest.mark.parametrize("recipe", [ln.QUARTET2, ln.TETRAJET2], ids=["quartet2", "tetrajet2"])
+@pytest.mark.parametrize("recipe", [ln.QUARTET2, ln.TETRAJET2, ln.NVIDIA], ids=["quartet2", "tetrajet2", "nvidia"])
 def test_quartet2_backward_is_unbiased_in_the_mean(recipe):
     M, N, K = 128, 128, 256
     d = syn.linear_quartet2(M, N, K, 4)
@@ -141,3 +141,18 @@ def test_ms_eden_backward_beats_sr_backward():
         err[name] = e
     assert err["eden"][0] < 0.7 * err["sr"][0]
     assert err["eden"][1] < 0.7 * err["sr"][1]
+
+
+def test_nvidia_recipe_reuses_the_forward_weights():
+    """The NVIDIA recipe's dX GEMM multiplies by the forward Q(W) itself
+    (square blocks, transposed), so with SR on dY the mean over seeds
+    converges to dY Q(W) and the re-used operand equals Q(W^T) quantised
+    directly from W^T."""
+    M, N, K = 128, 128, 256
+    d = syn.linear_quartet2(M, N, K, 8)
+    X, W, dY = (syn.bf16_bits_to_f32(d[k]) for k in ("X", "W", "dY"))
+    _, _, ctx = ln.linear_fwd(X, W, ln.NVIDIA)
+    ops = ln.bwd_operands(dY, ctx, ln.NVIDIA, 3)
+    direct = qn.quantize(W, qn.NVFP4, qn.RTN_SQUARE16, 0, transpose=True)
+    np.testing.assert_array_equal(ops["W_t"].codes, direct.codes)
+    np.testing.assert_array_equal(ops["W_t"].scales, direct.scales)
