@@ -231,6 +231,19 @@ def dequantize(qt, out_dtype=torch.float32, out=None):
     return out
 
 
+def transpose_square16(qt, linear=True, swizzled=True, out=None):
+    """fp4_transpose_square16: the transpose of a square-block quantised tensor."""
+    lib = load()
+    f = lib.fp4_transpose_square16
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.POINTER(fp4_qtensor), ctypes.POINTER(fp4_qtensor), ctypes.c_void_p]
+    if out is None:
+        out = alloc_qtensor(qt.cols, qt.rows, qt.fmt, linear, swizzled, device=qt.codes.device)
+    cin, cout = qt.c_struct(), out.c_struct()
+    _check(f(ctypes.byref(cin), ctypes.byref(cout), _stream()), "fp4_transpose_square16")
+    return out
+
+
 def hadamard(x, block, randomized=False, seed=0, sign_tag=0):
     lib = load()
     y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
@@ -262,13 +275,13 @@ def gemm(A, B, out_dtype=torch.float32, mask=None, inverse_had=0, out=None):
     return out
 
 
-RECIPE_QUARTET, RECIPE_QUARTET2, RECIPE_RTN, RECIPE_TETRAJET2 = 0, 1, 2, 3
+RECIPE_QUARTET, RECIPE_QUARTET2, RECIPE_RTN, RECIPE_TETRAJET2, RECIPE_NVIDIA = 0, 1, 2, 3, 4
 
 
 class fp4_recipe(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("fmt", "fwd_rounding", "fwd_had", "bwd_rounding", "bwd_had",
                                                "bwd_randomized", "mask_epilogue", "out_y", "out_dx",
-                                               "out_dw")]
+                                               "out_dw", "w_rounding", "w_reuse")]
 
 
 class fp4_ctx(ctypes.Structure):

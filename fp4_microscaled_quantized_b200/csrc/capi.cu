@@ -122,6 +122,43 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* codes, const uin
   }
 }
 
+// Transpose of FP4 codes (rows x cols, 2 per byte) in 64 x 64 tiles: the
+// tile's 64 input rows x 32 bytes are read as 8-byte chunks (coalesced),
+// spread to one code per byte in shared memory, and written back as 64
+// output rows x 32 bytes.
+__global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* in, int64_t rows, int64_t cols, uint8_t* out) {
+  __shared__ uint8_t tile[64][65];
+  const int64_t r0 = int64_t(blockIdx.y) * 64, c0 = int64_t(blockIdx.x) * 64;
+  const int t = threadIdx.x, tr = t >> 2, tc = (t & 3) * 16;      // one row, 16 codes
+  const uint2 w = *reinterpret_cast<const uint2*>(in + (r0 + tr) * (cols >> 1) + ((c0 + tc) >> 1));
+  const uint32_t ww[2] = {w.x, w.y};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) tile[tr][tc + j] = uint8_t((ww[j >> 3] >> (4 * (j & 7))) & 15u);
+  __syncthreads();
+  // output row c0 + tr, codes of input rows r0 + tc .. r0 + tc + 15
+  uint32_t o[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) o[j >> 3] |= uint32_t(tile[tc + j][tr]) << (4 * (j & 7));
+  *reinterpret_cast<uint2*>(out + (c0 + tr) * (rows >> 1) + ((r0 + tc) >> 1)) = make_uint2(o[0], o[1]);
+}
+
+// Scales of the transposed square-block tensor: output (r, k) (r an input
+// column, k a 16-group of input rows) takes the block scale of input block
+// (k, r / 16), i.e. input scale (16 k, r / 16); linear and/or tensor-core
+// layout.  Thread 0 also copies the tensor scale.
+__global__ void __launch_bounds__(256) k_transpose_sq16_scales(const uint8_t* in_sc, const float* in_ts, int64_t rows,
+                                                               int64_t cols, uint8_t* out_sc, uint8_t* out_swz,
+                                                               float* out_ts, int64_t nkb) {
+  const int64_t ng = rows >> 4, n = cols * ng;      // output: cols rows x rows/16 groups
+  if (blockIdx.x == 0 && threadIdx.x == 0) *out_ts = *in_ts;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / ng, k = i - r * ng;
+    const uint8_t v = in_sc[(k << 4) * (cols >> 4) + (r >> 4)];
+    if (out_sc) out_sc[i] = v;
+    if (out_swz) out_swz[swz_offset(r, k, nkb)] = v;
+  }
+}
+
 static int launch_pad(uint8_t* swz, int64_t rows, int64_t ng, cudaStream_t s) {
   int64_t nkb = (ng + 3) / 4;
   if (!swz || ((rows % 128) == 0 && (ng % 4) == 0)) return FP4_OK;
@@ -325,6 +362,29 @@ int fp4_dequantize(const fp4_qtensor* in, void* D, int32_t out_dtype, fp4_stream
     k_dequant<1><<<unsigned(blocks), 256, 0, s>>>(in->codes, in->scales, in->tensor_scale, in->fmt, in->rows, in->cols, D);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? FP4_OK : FP4_ERR_CUDA;
+}
+
+int fp4_transpose_square16(const fp4_qtensor* in, fp4_qtensor* out, fp4_stream_t stream) {
+  if (!in || !out || in->fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (in->rows < 0 || in->cols < 0 || in->rows % 64 || in->cols % 64) return FP4_ERR_INVALID_ARG;
+  out->rows = in->cols; out->cols = in->rows; out->fmt = FP4_NVFP4;
+  if (in->rows == 0 || in->cols == 0) return FP4_OK;
+  if (!in->codes || !in->scales || !in->tensor_scale) return FP4_ERR_INVALID_ARG;
+  int st = check_out(out);
+  if (st) return st;
+  if (!aligned(in->codes, 16)) return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dim3 grid(unsigned(in->cols / 64), unsigned(in->rows / 64));
+  k_transpose_codes<<<grid, 256, 0, s>>>(in->codes, in->rows, in->cols, out->codes);
+  count_launch();
+  const int64_t ng = in->rows / 16, n = in->cols * ng, nkb = (ng + 3) / 4;
+  int64_t blocks = (n + 255) / 256, cap = int64_t(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  k_transpose_sq16_scales<<<unsigned(blocks), 256, 0, s>>>(in->scales, in->tensor_scale, in->rows, in->cols,
+                                                           out->scales, out->scales_swz, out->tensor_scale, nkb);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return FP4_ERR_CUDA;
+  return launch_pad(out->scales_swz, out->rows, ng, s);
 }
 
 int fp4_hadamard(const void* x, float* y, int64_t rows, int64_t cols, fp4_had had, uint64_t seed,

@@ -48,7 +48,8 @@ size_t quant_ws_bwd(const fp4_recipe* r, int64_t M, int64_t N, int64_t K) {
 
 size_t quant_ws_fwd(const fp4_recipe* r, int64_t M, int64_t N, int64_t K) {
   size_t a = fp4_quantize_workspace_size(M, K, r->fmt, r->fwd_rounding, r->fwd_had);
-  size_t b = fp4_quantize_workspace_size(N, K, r->fmt, r->fwd_rounding, r->fwd_had);
+  const int w_rnd = r->w_rounding >= 0 ? r->w_rounding : r->fwd_rounding;
+  size_t b = fp4_quantize_workspace_size(N, K, r->fmt, w_rnd, r->fwd_had);
   return a256(a > b ? a : b);
 }
 
@@ -58,6 +59,8 @@ bool recipe_ok(const fp4_recipe* r) {
   if (r->out_y < 0 || r->out_y > 1 || r->out_dx < 0 || r->out_dx > 1 || r->out_dw < 0 || r->out_dw > 1)
     return false;
   if (r->mask_epilogue && (r->fwd_rounding != FP4_QUEST || r->fwd_had != 32)) return false;
+  if (r->w_rounding < -1 || r->w_rounding > FP4_RTN_SQUARE16) return false;
+  if (r->w_reuse && (r->w_rounding != FP4_RTN_SQUARE16 || r->fmt != FP4_NVFP4 || r->mask_epilogue)) return false;
   return true;
 }
 
@@ -69,16 +72,19 @@ int fp4_recipe_preset(int32_t id, fp4_recipe* r) {
   if (!r) return FP4_ERR_INVALID_ARG;
   switch (id) {
     case FP4_RECIPE_QUARTET:
-      *r = fp4_recipe{FP4_MXFP4, FP4_QUEST, 32, FP4_SR, 32, 1, 1, 0, 0, 0};
+      *r = fp4_recipe{FP4_MXFP4, FP4_QUEST, 32, FP4_SR, 32, 1, 1, 0, 0, 0, -1, 0};
       return FP4_OK;
     case FP4_RECIPE_QUARTET2:
-      *r = fp4_recipe{FP4_NVFP4, FP4_FOUR_OVER_SIX, 0, FP4_MS_EDEN, 128, 1, 0, 0, 0, 0};
+      *r = fp4_recipe{FP4_NVFP4, FP4_FOUR_OVER_SIX, 0, FP4_MS_EDEN, 128, 1, 0, 0, 0, 0, -1, 0};
       return FP4_OK;
     case FP4_RECIPE_RTN:
-      *r = fp4_recipe{FP4_NVFP4, FP4_RTN, 0, FP4_RTN, 0, 0, 0, 0, 0, 0};
+      *r = fp4_recipe{FP4_NVFP4, FP4_RTN, 0, FP4_RTN, 0, 0, 0, 0, 0, 0, -1, 0};
       return FP4_OK;
     case FP4_RECIPE_TETRAJET2:
-      *r = fp4_recipe{FP4_NVFP4, FP4_RTN, 0, FP4_SR, 128, 1, 0, 0, 0, 0};
+      *r = fp4_recipe{FP4_NVFP4, FP4_RTN, 0, FP4_SR, 128, 1, 0, 0, 0, 0, -1, 0};
+      return FP4_OK;
+    case FP4_RECIPE_NVIDIA:
+      *r = fp4_recipe{FP4_NVFP4, FP4_RTN, 0, FP4_SR, 16, 1, 0, 0, 0, 0, FP4_RTN_SQUARE16, 1};
       return FP4_OK;
     default:
       return FP4_ERR_INVALID_ARG;
@@ -102,7 +108,8 @@ int fp4_linear_fwd(const void* X, const void* W, int64_t M, int64_t N, int64_t K
   const fp4_had h{r->fwd_had, 0, 0};
   int st = fp4_quantize(X, M, K, 0, r->fmt, r->fwd_rounding, g, h, seed, TAG_X, &ctx->xq, ws, ws_bytes, s);
   if (st) return st;
-  st = fp4_quantize(W, N, K, 0, r->fmt, r->fwd_rounding, g, h, seed, TAG_W, &ctx->wq, ws, ws_bytes, s);
+  const int w_rnd = r->w_rounding >= 0 ? r->w_rounding : r->fwd_rounding;
+  st = fp4_quantize(W, N, K, 0, r->fmt, w_rnd, g, h, seed, TAG_W, &ctx->wq, ws, ws_bytes, s);
   if (st) return st;
   return fp4_gemm(&ctx->xq, &ctx->wq, Y, r->out_y, nullptr, 0, s);
 }
@@ -125,11 +132,20 @@ int fp4_linear_bwd(const void* dY, const fp4_ctx* ctx, int64_t M, int64_t N, int
   const int inv_h = r->mask_epilogue ? r->fwd_had : 0;
   int st;
   if (dX) {
-    const fp4_had h{r->bwd_had, rz, GEMM_DX};
-    st = fp4_quantize(dY, M, N, 0, r->fmt, r->bwd_rounding, g, h, step_seed, TAG_E_ROW, &e_row, qw, qws, s);
-    if (st) return st;
-    st = fp4_requantize(&ctx->wq, 1, r->bwd_rounding, h, step_seed, TAG_W_T, &w_t, qw, qws, s);
-    if (st) return st;
+    if (r->w_reuse) {
+      // the forward Q(W) itself, transposed; dY without a rotation to match it
+      const fp4_had h0{0, 0, GEMM_DX};
+      st = fp4_quantize(dY, M, N, 0, r->fmt, r->bwd_rounding, g, h0, step_seed, TAG_E_ROW, &e_row, qw, qws, s);
+      if (st) return st;
+      st = fp4_transpose_square16(&ctx->wq, &w_t, s);
+      if (st) return st;
+    } else {
+      const fp4_had h{r->bwd_had, rz, GEMM_DX};
+      st = fp4_quantize(dY, M, N, 0, r->fmt, r->bwd_rounding, g, h, step_seed, TAG_E_ROW, &e_row, qw, qws, s);
+      if (st) return st;
+      st = fp4_requantize(&ctx->wq, 1, r->bwd_rounding, h, step_seed, TAG_W_T, &w_t, qw, qws, s);
+      if (st) return st;
+    }
     st = fp4_gemm(&e_row, &w_t, dX, r->out_dx, r->mask_epilogue ? ctx->xq.mask : nullptr, inv_h, s);
     if (st) return st;
   }

@@ -130,6 +130,17 @@ size_t fp4_quantize_workspace_size(int64_t rows, int64_t cols, int32_t fmt,
  * out_dtype, cols not a multiple of the group), FP4_ERR_ALIGNMENT. */
 int fp4_dequantize(const fp4_qtensor *in, void *D_dev, int32_t out_dtype, fp4_stream_t stream);
 
+/* Transpose of a quantised tensor with 16 x 16 square-block scales
+ * (FP4_RTN_SQUARE16): out = in^T, codes transposed and each block's scale
+ * moved to the transposed block -- equal to quantising the transposed input
+ * directly, which is how the NVIDIA recipe re-uses Q(W) for W^T ([QII] "The
+ * square-block trade-off").  in: NVFP4, rows and cols multiples of 64 and
+ * 16, codes, linear scales and tensor scale (device).  out: caller-owned,
+ * codes (cols x rows/2), scales and/or scales_swz, tensor_scale; the call
+ * writes rows, cols, fmt.  The result is the transpose only when `in` has
+ * square-block scales.  Errors: FP4_ERR_INVALID_ARG, FP4_ERR_ALIGNMENT. */
+int fp4_transpose_square16(const fp4_qtensor *in, fp4_qtensor *out, fp4_stream_t stream);
+
 /* Bytes of the swizzled scale buffer for rows x n_groups scales. */
 size_t fp4_swizzled_scale_bytes(int64_t rows, int64_t n_groups);
 
@@ -236,6 +247,12 @@ int fp4_gemm(const fp4_qtensor *A, const fp4_qtensor *B, void *D_dev, int32_t ou
  *      backward de-quantise, transpose, RHT128 on the inner dimension and
  *      element-wise SR (the same graph as FP4_RECIPE_QUARTET2 with SR in
  *      place of MS-EDEN).
+ *  FP4_RECIPE_NVIDIA   the NVIDIA recipe [QII] describes ("The square-block
+ *      trade-off"): NVFP4; forward X with 1x16 RTN, W with 16x16
+ *      square-block RTN, no rotation; backward SR; the dX GEMM re-uses the
+ *      forward Q(W) transposed (fp4_transpose_square16) against SR(dY) without
+ *      a rotation; the dW GEMM uses the 16-point RHT on dY^T and on the
+ *      re-quantised X^T.
  * Seeds: every random draw of one backward step is keyed by step_seed; the
  * dX GEMM's operands share sign tag 0, the dW GEMM's sign tag 1; SR tensor
  * tags 1 (dY), 2 (W_q^T), 3 (dY^T), 4 (X_q^T); forward tags 5 (X), 6 (W). */
@@ -243,7 +260,8 @@ enum fp4_recipe_id {
   FP4_RECIPE_QUARTET = 0,
   FP4_RECIPE_QUARTET2 = 1,
   FP4_RECIPE_RTN = 2,
-  FP4_RECIPE_TETRAJET2 = 3
+  FP4_RECIPE_TETRAJET2 = 3,
+  FP4_RECIPE_NVIDIA = 4
 };
 
 typedef struct {
@@ -255,6 +273,11 @@ typedef struct {
   int32_t bwd_randomized; /* 1: RHT (random signs), 0: H                     */
   int32_t mask_epilogue;  /* 1: Quartet mask + H^-1 epilogue (fwd QuEST)     */
   int32_t out_y, out_dx, out_dw; /* 0 fp32, 1 bf16                           */
+  int32_t w_rounding;     /* fp4_rounding of W in the forward pass, or -1 for
+                             fwd_rounding (FP4_RTN_SQUARE16: square blocks)   */
+  int32_t w_reuse;        /* 1: the dX GEMM multiplies by the forward Q(W),
+                             transposed (needs w_rounding FP4_RTN_SQUARE16),
+                             and dY is quantised for it without a rotation    */
 } fp4_recipe;
 
 /* Fill *r with a preset; returns FP4_ERR_INVALID_ARG for an unknown id. */

@@ -15,7 +15,8 @@ from oracle import quant as qn
 
 pytestmark = pytest.mark.gpu
 
-RECIPES = {"quartet": ln.QUARTET, "quartet2": ln.QUARTET2, "rtn": ln.RTN, "tetrajet2": ln.TETRAJET2}
+RECIPES = {"quartet": ln.QUARTET, "quartet2": ln.QUARTET2, "rtn": ln.RTN, "tetrajet2": ln.TETRAJET2,
+           "nvidia": ln.NVIDIA}
 
 
 def dev(bits):
@@ -44,7 +45,7 @@ def check_ctx(g, o):
 def data(name, M, N, K, seed):
     if name == "quartet":
         return syn.linear_quartet(M, N, K, seed)
-    if name in ("quartet2", "tetrajet2"):
+    if name in ("quartet2", "tetrajet2", "nvidia"):
         return syn.linear_quartet2(M, N, K, seed)
     d = syn.linear_rtn_small(seed) if (M, N, K) == (256, 512, 512) else {
         "X": syn.gaussian((M, K), 1.0, seed, 0), "W": syn.gaussian((N, K), 0.02, seed, 1)}
@@ -67,11 +68,13 @@ def test_config1_rtn_forward(cuda_lib):
 @pytest.mark.parametrize("name,M,N,K", [("quartet", 384, 256, 512), ("quartet2", 512, 384, 256),
                                         ("rtn", 256, 128, 256), ("quartet", 256, 512, 256),
                                         ("quartet2", 256, 128, 512), ("tetrajet2", 384, 256, 512),
-                                        ("tetrajet2", 256, 384, 256)])
+                                        ("tetrajet2", 256, 384, 256), ("nvidia", 256, 384, 512),
+                                        ("nvidia", 384, 256, 256)])
 def test_linear_fwd_bwd_parity(cuda_lib, name, M, N, K):
     d = data(name, M, N, K, 3)
     preset = {"quartet": cuda_lib.RECIPE_QUARTET, "quartet2": cuda_lib.RECIPE_QUARTET2,
-              "rtn": cuda_lib.RECIPE_RTN, "tetrajet2": cuda_lib.RECIPE_TETRAJET2}[name]
+              "rtn": cuda_lib.RECIPE_RTN, "tetrajet2": cuda_lib.RECIPE_TETRAJET2,
+              "nvidia": cuda_lib.RECIPE_NVIDIA}[name]
     r = cuda_lib.recipe(preset)
     Y, ctx = cuda_lib.linear_fwd(dev(d["X"]), dev(d["W"]), r, seed=0)
     step = 1234

@@ -252,3 +252,19 @@ def test_square_block_argument_errors(cuda_lib):
         with pytest.raises(cuda_lib.Fp4Error) as e:
             cuda_lib.quantize(y, fmt, qn.RTN_SQUARE16, had)
         assert e.value.status == 2
+
+
+@pytest.mark.parametrize("shape", [(64, 128), (256, 512), (640, 192)])
+def test_transpose_square16(cuda_lib, shape):
+    """fp4_transpose_square16 against the oracle's transpose of the same
+    square-block quantised tensor (codes, linear and tensor-core scales,
+    tensor scale), and equal to quantising the transposed input directly."""
+    bits = syn.outlier_elements(shape, seed=17, stream=shape[1])
+    x = syn.bf16_bits_to_f32(bits)
+    q = cuda_lib.quantize(to_dev(bits), qn.NVFP4, qn.RTN_SQUARE16, 0)
+    t = cuda_lib.transpose_square16(q)
+    o = qn.transpose_square16(qn.quantize(x, qn.NVFP4, qn.RTN_SQUARE16, 0))
+    assert_qt_equal(t, o)
+    d = cuda_lib.quantize(to_dev(bits), qn.NVFP4, qn.RTN_SQUARE16, 0, transpose=True)
+    torch.cuda.synchronize()
+    assert torch.equal(t.codes, d.codes) and torch.equal(t.scales, d.scales)
