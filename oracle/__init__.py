@@ -20,6 +20,6 @@ anything here, and nothing here imports the product path.
 Arithmetic contract (shared by definition, not by code, with the GPU path):
 quantizer arithmetic is IEEE fp32 with round-to-nearest-even on every
 operation (numpy float32 ops, no fused multiply-add), division is correctly
-rounded, sums are fixed pairwise trees, maxima are exact; GEMM references
-are fp64.
+rounded, sums are fixed pairwise trees (float64 in the MSE search's
+tensor-scale step), maxima are exact; GEMM references are fp64.
 """

@@ -1,5 +1,6 @@
 """Micro-scaled FP4 quantizers: MXFP4 / NVFP4 x {RTN, QuEST, Four-Over-Six,
-SR, MS-EDEN}, plus dequantisation and the tensor-core scale layout.
+SR, MS-EDEN}, NVFP4 square-block RTN and the MSE-optimal scale search, plus
+dequantisation and the tensor-core scale layout.
 
 Test infrastructure only (see ``oracle/__init__.py``).
 
@@ -244,6 +245,94 @@ def nvfp4_quest(x, amax=None):
     mask = (np.abs(v) > F32(6.0)) & ok[..., None]
     return QTensor(codes.reshape(x.shape), s8, s32, NVFP4,
                    mask=mask.reshape(x.shape))
+
+
+def pairwise_sum_f64(v):
+    """Sum of a 1-D array in float64 as a fixed pairwise tree over its order,
+    padded with zeros to a power of two (the padding length does not change
+    the value)."""
+    a = np.asarray(v, dtype=np.float64).reshape(-1)
+    n = 1
+    while n < a.size:
+        n <<= 1
+    a = np.concatenate([a, np.zeros(n - a.size)])
+    while a.size > 1:
+        a = a[0::2] + a[1::2]
+    return np.float64(a[0]) if a.size else np.float64(0.0)
+
+
+def mse_group_scales(xg, s_T):
+    """The group step of the MSE-optimal scale search ("Bridging the Gap
+    Between Promise and Performance for Microscaling FP4 Quantization" page,
+    "MSE-Optimized Grid and Scale Selection"): with the
+    tensor scale s_T held, each 16-element group takes the E4M3 scale code c
+    (1..126) whose RTN codes give the smallest squared error, the error of a
+    candidate being the fp32 pairwise sum of fp32((x - fp32(q d))^2) with
+    d = fp32(E4M3(c) s_T).  READINGS: the "1-D line search" visits every
+    finite non-zero E4M3 code; ties keep the larger scale; a group whose
+    maximum is zero takes code 0 (all codes zero), as under RTN."""
+    gmax = _group_max(xg)
+    best_c = np.zeros(gmax.shape, dtype=np.int64)
+    best_e = np.full(gmax.shape, np.inf, dtype=F32)
+    for c in range(1, 127):
+        dd = np.full(gmax.shape, F32(F32(fm.E4M3_VALUES[c]) * F32(s_T)), dtype=F32)
+        codes, _, _ = _encode_rtn(xg, dd)
+        e = _sse(xg, codes, dd)
+        better = e <= best_e                     # ascending scale: ties go to the larger
+        best_c = np.where(better, c, best_c)
+        best_e = np.where(better, e, best_e).astype(F32)
+    return np.where(gmax > 0, best_c, 0).astype(np.uint8)
+
+
+def mse_tensor_scale(x, s8, codes, s_T):
+    """The tensor-scale step: with the group scale codes and the element codes
+    held, the de-quantised tensor is s_T * u with u = E4M3(c_j) q_i, and the
+    squared error is smallest at s_T = <x, u> / <u, u>.  READING: the page's
+    second 1-D search is this closed-form least-squares solution; both inner
+    products are float64 pairwise trees over the row-major element order
+    (every product is exact in float64), the quotient is rounded once to
+    fp32, and s_T is kept when either sum is not positive or the quotient is
+    not a finite positive fp32 value."""
+    u = (fm.e4m3_value(s8).astype(np.float64)[..., None]
+         * fm.decode_e2m1(codes).astype(np.float64).reshape(s8.shape + (16,)))
+    x64 = np.asarray(x, dtype=F32).astype(np.float64).reshape(u.shape)
+    num = pairwise_sum_f64(x64 * u)
+    den = pairwise_sum_f64(u * u)
+    if not (num > 0 and den > 0):
+        return F32(s_T)
+    with np.errstate(over="ignore"):
+        t = F32(num / den)
+    return t if (np.isfinite(t) and t > 0) else F32(s_T)
+
+
+def nvfp4_mse_search(x, iters):
+    """NVFP4 with MSE-optimal scales by alternating optimisation ("Bridging
+    the Gap Between Promise and Performance for Microscaling FP4 Quantization"
+    page, "MSE-Optimized Grid and Scale Selection", NVFP4 without rotations):
+    start from the RTN tensor scale amax / (6 * 256); a
+    group step; then `iters` times a tensor-scale step followed by a group
+    step.  The codes are RTN_E2M1(x * fp32(1/d)) at the final scales.  Each
+    step lowers (or keeps) the exact squared error, so the error does not
+    grow with `iters`.  Returns the QTensor and the tensor scale after each
+    step in ``extra["s_T"]``."""
+    x = np.asarray(x, dtype=F32)
+    amax = abs_max(x)
+    s_T = nvfp4_tensor_scale(amax, NV_RTN_DIV)
+    xg = _groups(x, 16)
+    history = [s_T]
+
+    def group_step(s_T):
+        s8 = mse_group_scales(xg, s_T)
+        d = (fm.e4m3_value(s8).astype(F32) * F32(s_T)).astype(F32)
+        codes, _, _ = _encode_rtn(xg, d)
+        return s8, codes
+
+    s8, codes = group_step(s_T)
+    for _ in range(iters):
+        s_T = mse_tensor_scale(x, s8, codes, s_T)
+        history.append(s_T)
+        s8, codes = group_step(s_T)
+    return QTensor(codes.reshape(x.shape), s8, F32(s_T), NVFP4, extra={"s_T": history})
 
 
 def ms_eden_pass1(y, chunk):

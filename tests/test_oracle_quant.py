@@ -375,3 +375,112 @@ def test_square_block_quantisation_commutes_with_transpose():
     np.testing.assert_array_equal(b.codes, a.codes.T)
     np.testing.assert_array_equal(b.scales, np.repeat(a.scales[::16].T, 16, axis=0))
     assert b.tensor_scale == a.tensor_scale
+
+
+# ------------------------------- MSE-optimal scale search (alternating) ----
+def _group_sse32(x, qt, s_T=None):
+    """Per-group fp32 squared error of a QTensor, the search's own measure."""
+    xg = x.reshape(x.shape[0], -1, 16)
+    d = (fm.e4m3_value(qt.scales).astype(F32) * F32(qt.tensor_scale if s_T is None else s_T)).astype(F32)
+    return qn._sse(xg, qt.codes.reshape(xg.shape), d)
+
+
+def test_mse_search_never_worse_than_rtn_or_four_over_six():
+    """The group step's candidates include the RTN scale and both
+    Four-Over-Six candidates (same tensor scale), so no group's error can
+    be larger than theirs."""
+    rng = np.random.default_rng(21)
+    x = (rng.standard_t(3, (48, 256)) * np.exp(rng.uniform(-3, 3, (48, 1)))).astype(F32)
+    m = qn.nvfp4_mse_search(x, 0)
+    r, f = qn.nvfp4_rtn(x), qn.nvfp4_four_over_six(x)
+    assert m.tensor_scale == r.tensor_scale == f.tensor_scale
+    em, er, ef = _group_sse32(x, m), _group_sse32(x, r), _group_sse32(x, f)
+    assert np.all(em <= er) and np.all(em <= ef)
+    assert np.mean(em < ef) > 0.3                  # and strictly better on many groups
+
+
+def test_mse_search_brute_force():
+    """Pure-python search over all 126 E4M3 scales in float64: the chosen
+    scale's error is the minimum (up to fp32 rounding of near ties)."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal((8, 16 * 6)) * np.exp(rng.uniform(-2, 2, (8, 1)))).astype(F32)
+    x[:, 5::16] *= 5                                  # an outlier per group
+    qt = qn.nvfp4_mse_search(x, 0)
+    s_T = float(qt.tensor_scale)
+    assert s_T == float(F32(F32(np.max(np.abs(x))) / F32(1536.0)))
+    for r in range(x.shape[0]):
+        for g in range(6):
+            xs = [float(v) for v in x[r, 16 * g:16 * g + 16]]
+            errs = [_py_sse(xs, float(F32(fm.E4M3_VALUES[c] * F32(s_T)))) for c in range(1, 127)]
+            best = min(errs)
+            got = errs[int(qt.scales[r, g]) - 1]
+            assert got <= best * (1 + 1e-5) + 1e-30
+            # the chosen scale is the largest among the (near-)minimisers
+            assert all(e > best * (1 + 1e-5) for e in errs[int(qt.scales[r, g]):]) or got == best
+
+
+def test_mse_search_lossless_on_grid_values():
+    """x = 2^k E4M3(c_j) q_i with a 256 scale setting amax: the RTN tensor
+    scale is 2^k, some candidate reproduces every group exactly, and the
+    tensor-scale step keeps 2^k (<x, u> = 2^k <u, u> exactly)."""
+    rng = np.random.default_rng(23)
+    k = -6
+    codes = rng.integers(0, 16, (4, 64)).astype(np.uint8)
+    codes[:, ::16] = 7
+    s8 = rng.integers(8, 120, (4, 4)).astype(np.uint8)
+    s8[0, 0] = 0x78
+    vals = fm.decode_e2m1(codes).astype(np.float64) * (fm.e4m3_value(s8) * 2.0 ** k).repeat(16, -1)
+    for iters in (0, 2):
+        qt = qn.nvfp4_mse_search(vals.astype(F32), iters)
+        assert float(qt.tensor_scale) == 2.0 ** k
+        np.testing.assert_array_equal(qn.dequant_f64(qt), vals)
+
+
+def test_mse_search_error_does_not_grow_with_iterations():
+    """Each alternation lowers or keeps the exact squared error."""
+    rng = np.random.default_rng(24)
+    x = (rng.standard_t(3, (32, 512)) * 0.02).astype(F32)
+    errs = []
+    for iters in range(4):
+        qt = qn.nvfp4_mse_search(x, iters)
+        errs.append(float(np.sum((qn.dequant_f64(qt) - x.astype(np.float64)) ** 2)))
+        assert len(qt.extra["s_T"]) == iters + 1
+    for a, b in zip(errs, errs[1:]):
+        assert b <= a * (1 + 1e-6)
+    assert errs[-1] < errs[0]
+
+
+def test_mse_tensor_scale_step_is_the_least_squares_minimiser():
+    """With the codes held, the step's s_T minimises sum (x - s u)^2: the
+    error at s_T is below the error at s_T (1 +- 2^-12), and the derivative
+    2 sum u (s u - x) vanishes to rounding."""
+    rng = np.random.default_rng(25)
+    x = (rng.standard_normal((16, 256)) * 3.0).astype(F32)
+    q0 = qn.nvfp4_mse_search(x, 0)
+    s_new = float(qn.mse_tensor_scale(x, q0.scales, q0.codes.reshape(16, 16, 16), q0.tensor_scale))
+    u = (fm.e4m3_value(q0.scales).astype(np.float64)[..., None]
+         * fm.decode_e2m1(q0.codes).astype(np.float64).reshape(16, 16, 16)).reshape(-1)
+    xv = x.astype(np.float64).reshape(-1)
+    err = lambda s: float(np.sum((xv - s * u) ** 2))
+    assert err(s_new) < err(s_new * (1 + 2.0 ** -12)) and err(s_new) < err(s_new * (1 - 2.0 ** -12))
+    assert abs(float(np.dot(u, s_new * u - xv))) <= 1e-6 * float(np.dot(np.abs(u), np.abs(xv)))
+
+
+def test_mse_search_degenerate_inputs():
+    z = np.zeros((2, 32), dtype=F32)
+    qt = qn.nvfp4_mse_search(z, 3)
+    assert float(qt.tensor_scale) == 1.0 and not qt.scales.any() and not qt.codes.any()
+    x = np.zeros((2, 32), dtype=F32)
+    x[1, 20] = -3.0                                    # one non-zero group
+    qt = qn.nvfp4_mse_search(x, 1)
+    assert qt.scales[0, 0] == qt.scales[0, 1] == qt.scales[1, 0] == 0
+    np.testing.assert_array_equal(qn.dequant_f64(qt), x.astype(np.float64))
+
+
+def test_pairwise_sum_f64_padding_invariant():
+    v = np.random.default_rng(26).standard_normal(1000) * np.exp(np.random.default_rng(27).uniform(-20, 20, 1000))
+    a = qn.pairwise_sum_f64(v)
+    b = qn.pairwise_sum_f64(np.concatenate([v, np.zeros(3096)]))
+    assert a == b
+    assert a == pytest.approx(math.fsum(v), rel=1e-12, abs=1e-300)
+    assert qn.pairwise_sum_f64([1.0, 2.0, 3.0]) == 6.0
