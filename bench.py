@@ -362,6 +362,9 @@ def sweep_cases(api):
                 rand = rnd in (api.SR, api.MS_EDEN) and had > 0
                 out.append(("%s-%s-h%d" % (fname, RND_NAMES[rnd], had), fmt, rnd, had, rand))
     out.append(("nvfp4-rtn16x16-h0", api.NVFP4, api.RTN_SQUARE16, 0, False))
+    # the MSE-optimal scale search (fp4_quantize_mse) with 0 and 2 alternations
+    out.append(("nvfp4-mse-i0-h0", api.NVFP4, "mse0", 0, False))
+    out.append(("nvfp4-mse-i2-h0", api.NVFP4, "mse2", 0, False))
     return out
 
 
@@ -369,7 +372,11 @@ def sweep_bytes_per_elem(api, fmt, rnd, had):
     """Algorithmic HBM bytes per element of one quantise call: bf16 read 2 B,
     codes 0.5, one scale copy 1/g; NVFP4 global-scale modes read the input
     twice (amax or 16 x 16 block-maximum pass); QuEST writes a 1-bit mask; MS-EDEN writes and re-reads
-    bf16 pseudo-scales (2 x 2/16) and fp32 EDEN factors (2 x 4/had)."""
+    bf16 pseudo-scales (2 x 2/16) and fp32 EDEN factors (2 x 4/had).  The
+    MSE search ("mseI", I alternations) reads the input once for the amax and
+    once per group step, writing codes and scales each time."""
+    if isinstance(rnd, str):
+        return 2.0 + (int(rnd[3:]) + 1) * (2.0 + 0.5 + 1.0 / 16)
     g = api.GROUP[fmt]
     b = 2.0 + 0.5 + 1.0 / g
     if fmt == api.NVFP4 and rnd != api.MS_EDEN:
@@ -412,8 +419,12 @@ def quant_sweep(args):
         for name, fmt, rnd, had, rand in cases:
             out = api.alloc_qtensor(rows, SWEEP_COLS, fmt, linear=False, mask=(rnd == api.QUEST),
                                     device=dev)
-            ws = api.alloc_workspace(api.workspace_size(rows, SWEEP_COLS, fmt, rnd, had), dev)
-            call = lambda s: api.quantize(x, fmt, rnd, had, rand, s, 0, 1, out=out, ws=ws)  # noqa: E731
+            if isinstance(rnd, str):
+                ws = api.alloc_workspace(api.quantize_mse_workspace_size(rows, SWEEP_COLS), dev)
+                call = lambda s, it=int(rnd[3:]): api.quantize_mse(x, it, out=out, ws=ws)  # noqa: E731
+            else:
+                ws = api.alloc_workspace(api.workspace_size(rows, SWEEP_COLS, fmt, rnd, had), dev)
+                call = lambda s: api.quantize(x, fmt, rnd, had, rand, s, 0, 1, out=out, ws=ws)  # noqa: E731
             lc0 = api.launch_count()
             for w in range(3):
                 call(w)

@@ -231,6 +231,34 @@ def dequantize(qt, out_dtype=torch.float32, out=None):
     return out
 
 
+def quantize_mse_workspace_size(rows, cols):
+    lib = load()
+    f = lib.fp4_quantize_mse_workspace_size
+    f.restype = ctypes.c_size_t
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    return f(rows, cols)
+
+
+def quantize_mse(x, iters=0, linear=True, swizzled=True, out=None, ws=None):
+    """fp4_quantize_mse: NVFP4 with MSE-optimal group scales and `iters`
+    least-squares tensor-scale updates; returns a QTensor."""
+    lib = load()
+    f = lib.fp4_quantize_mse
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                  ctypes.POINTER(fp4_qtensor), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
+    rows, cols = x.shape
+    if out is None:
+        out = alloc_qtensor(rows, cols, NVFP4, linear, swizzled, device=x.device)
+    if ws is None:
+        ws = alloc_workspace(quantize_mse_workspace_size(rows, cols), x.device)
+    cs = out.c_struct()
+    _check(f(_ptr(x), rows, cols, int(iters), ctypes.byref(cs), _ptr(ws), ws.numel(), _stream()),
+           "fp4_quantize_mse")
+    return out
+
+
 def transpose_square16(qt, linear=True, swizzled=True, out=None):
     """fp4_transpose_square16: the transpose of a square-block quantised tensor."""
     lib = load()

@@ -5,6 +5,7 @@
 
 #include "../../include/fp4.h"
 #include "quant_dispatch.cuh"
+#include "quant_mse.cuh"
 
 namespace fp4 {
 
@@ -342,6 +343,48 @@ int fp4_requantize(const fp4_qtensor* in, int32_t transpose, int32_t rounding, f
   p.randomized = had.randomized ? 1 : 0;
   return run_quant(transpose ? LD_TRANS_FP4 : LD_ROW_FP4, fmt, rounding, had.block, p, ws,
                    ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t fp4_quantize_mse_workspace_size(int64_t rows, int64_t cols) {
+  if (rows < 0 || cols < 0 || cols % 32) return 0;
+  return 256 + align256(size_t(mse_blocks(rows, cols)) * sizeof(double2));
+}
+
+int fp4_quantize_mse(const void* x, int64_t rows, int64_t cols, int32_t iters, fp4_qtensor* out, void* ws,
+                     size_t ws_bytes, fp4_stream_t stream) {
+  if (rows < 0 || cols < 0 || cols % 32 || iters < 0 || iters > 64 || !out) return FP4_ERR_INVALID_ARG;
+  out->rows = rows; out->cols = cols; out->fmt = FP4_NVFP4;
+  if (rows == 0 || cols == 0) return FP4_OK;
+  int st = check_out(out);
+  if (st) return st;
+  if (!x) return FP4_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return FP4_ERR_ALIGNMENT;
+  const size_t need = fp4_quantize_mse_workspace_size(rows, cols);
+  if (!ws || ws_bytes < need) return FP4_ERR_WORKSPACE;
+  if (!aligned(ws, 16)) return FP4_ERR_ALIGNMENT;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  QParams p{};
+  p.x = x; p.in_rows = rows; p.in_cols = cols; p.rows = rows; p.cols = cols;
+  p.amax_bits = reinterpret_cast<uint32_t*>(w);
+  p.status = status_ptr();
+  p.nkb = ((cols / 16) + 3) / 4;
+  if (cudaMemsetAsync(p.amax_bits, 0, sizeof(uint32_t), s) != cudaSuccess) return FP4_ERR_CUDA;
+  if (launch_quant<LD_ROW>(FP4_NVFP4, R_AMAX, 0, p, s) != cudaSuccess) return FP4_ERR_CUDA;
+  MseParams m{};
+  m.x = static_cast<const uint16_t*>(x); m.rows = rows; m.cols = cols;
+  m.codes = out->codes; m.scales = out->scales; m.swz = out->scales_swz; m.nkb = p.nkb;
+  m.ts = out->tensor_scale; m.amax_bits = p.amax_bits;
+  m.partial = reinterpret_cast<double2*>(w + 256);
+  m.status = p.status;
+  m.first = 1;
+  if (launch_mse_group(m, s) != cudaSuccess) return FP4_ERR_CUDA;
+  m.first = 0;
+  for (int i = 0; i < iters; ++i) {
+    if (launch_mse_tensor(m.partial, mse_blocks(rows, cols), m.ts, s) != cudaSuccess) return FP4_ERR_CUDA;
+    if (launch_mse_group(m, s) != cudaSuccess) return FP4_ERR_CUDA;
+  }
+  return launch_pad(out->scales_swz, rows, cols / 16, s);
 }
 
 int fp4_dequantize(const fp4_qtensor* in, void* D, int32_t out_dtype, fp4_stream_t stream) {

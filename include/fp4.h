@@ -10,7 +10,8 @@
  *        Four-Over-Six, MS-EDEN (Algorithm 1) and its post hoc range
  *        alignment, the Quartet II computation graph;
  *  [BG]  "Bridging the Gap Between Promise and Performance for Microscaling
- *        FP4 Quantization" -- MXFP4 / NVFP4 formats.
+ *        FP4 Quantization" -- MXFP4 / NVFP4 formats, the MSE-optimal
+ *        alternating scale search.
  *
  * Conventions for every call
  *  - All pointers named *_dev, and every pointer inside fp4_qtensor, are
@@ -140,6 +141,33 @@ int fp4_dequantize(const fp4_qtensor *in, void *D_dev, int32_t out_dtype, fp4_st
  * writes rows, cols, fmt.  The result is the transpose only when `in` has
  * square-block scales.  Errors: FP4_ERR_INVALID_ARG, FP4_ERR_ALIGNMENT. */
 int fp4_transpose_square16(const fp4_qtensor *in, fp4_qtensor *out, fp4_stream_t stream);
+
+/* NVFP4 quantisation with MSE-optimal scales by alternating optimisation
+ * ([BG] "MSE-Optimized Grid and Scale Selection", NVFP4 without rotation).
+ *  1. s_T = amax / (6 * 256), the RTN tensor scale (1 for an all-zero x).
+ *  2. Group step: each 16-element group takes the E4M3 scale code c in
+ *     1..126 whose RTN codes of x * fp32(1 / d), d = fp32(E4M3(c) * s_T),
+ *     give the smallest fp32 squared error (pairwise tree of
+ *     fp32((x - fp32(q d))^2)); ties keep the larger c; a group whose
+ *     maximum is zero takes c = 0 and zero codes.
+ *  3. `iters` times: the tensor-scale step s_T = fp32(<x, u> / <u, u>) with
+ *     u = E4M3(c_group) * q, the closed-form least-squares tensor scale for
+ *     the codes held (both sums float64 pairwise trees over the row-major
+ *     element order; s_T is kept when a sum is not positive or the quotient
+ *     is not a finite positive fp32 value), then the group step again.
+ * The squared error does not grow with `iters`.  x_dev: bf16 rows x cols,
+ * row-major, 16-byte aligned; cols a multiple of 32.  iters: 0..64.  out:
+ * as for fp4_quantize (codes, scales and/or scales_swz, tensor_scale = the
+ * final s_T; mask unused); the call writes rows, cols and fmt = NVFP4.
+ * ws_dev: fp4_quantize_mse_workspace_size bytes, 16-byte aligned: the amax
+ * word at byte 0, then one float64 pair per 8192 elements at byte 256.
+ * Launches 2 + 2 * iters kernels (plus one when the swizzled scales need
+ * padding).  A non-finite input sets FP4_ERR_NONFINITE_INPUT on the device.
+ * Errors: FP4_ERR_INVALID_ARG (shape, iters, null pointers),
+ * FP4_ERR_ALIGNMENT, FP4_ERR_WORKSPACE. */
+size_t fp4_quantize_mse_workspace_size(int64_t rows, int64_t cols);
+int fp4_quantize_mse(const void *x_dev, int64_t rows, int64_t cols, int32_t iters,
+                     fp4_qtensor *out, void *ws_dev, size_t ws_bytes, fp4_stream_t stream);
 
 /* Bytes of the swizzled scale buffer for rows x n_groups scales. */
 size_t fp4_swizzled_scale_bytes(int64_t rows, int64_t n_groups);
