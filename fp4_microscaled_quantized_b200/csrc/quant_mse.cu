@@ -6,6 +6,8 @@
 // rounded reciprocal (a per-block table, s_T being uniform), the RTN codes of
 // x * (1/d) and their fp32 squared error (sse16, the pairwise tree of
 // fp32((x - fp32(q d))^2)); the smallest error wins, ties to the larger code.
+// Candidates that the top element's own error term already rules out are not
+// evaluated in full (top_term); the result is that of the exhaustive scan.
 // A group whose maximum is zero (or NaN) takes code 0 and zero codes.  With
 // the winning codes, u = E4M3(c) q is exact in fp32 and x u, u u are exact in
 // float64; the block sums both over its 8192 consecutive elements as a
@@ -30,6 +32,44 @@ __device__ __forceinline__ double tree16d(const double* v) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) b[i] = __dadd_rn(a[2 * i], a[2 * i + 1]);
   return __dadd_rn(__dadd_rn(b[0], b[1]), __dadd_rn(b[2], b[3]));
+}
+
+// A value of the group whose magnitude is the group maximum (0 when none is,
+// e.g. a NaN maximum).
+__device__ __forceinline__ float top_value(const float* x, float gm) {
+  float t = 0.0f;
+#pragma unroll
+  for (int j = 15; j >= 0; --j) t = fabsf(x[j]) == gm ? x[j] : t;
+  return t;
+}
+
+// The candidate's squared-error term of one element, computed exactly as the
+// candidate's group error computes it (code of fp32(x * inv) by the same
+// conversion, zero when the scale is unusable; fp32((x - fp32(q d))^2)).  The
+// group error is a round-to-nearest pairwise sum of non-negative terms, which
+// is never smaller than any one of them, so a candidate whose top-element term
+// exceeds the best error found so far cannot be the minimiser.
+__device__ __forceinline__ float top_term(float xt, float d, float inv, bool ok) {
+  const uint32_t code = ok ? (e2m1x2_rn(__fmul_rn(xt, inv), 0.0f) & 0xFu) : 0u;
+  const float q = __half2float(__ushort_as_half(uint16_t(e2m1x2_to_f16x2(code) & 0xFFFFu)));
+  const float e = __fsub_rn(xt, __fmul_rn(q, d));
+  return __fmul_rn(e, e);
+}
+
+// E4M3 code nearest gm / (6 s_T), clamped to 1..126 (only a visiting order).
+__device__ __forceinline__ int seed_code(float gm, float inv6) {
+  const int c = int(e4m3_rtn(__fmul_rn(gm, inv6)));
+  return c < 1 ? 1 : (c > 126 ? 126 : c);
+}
+
+// Full error of candidate c for one group; the smaller error wins, a tie goes
+// to the larger code -- the result of an ascending scan with <=, whatever the
+// order candidates are visited in.  NaN errors never win.
+__device__ __forceinline__ void consider(const float* xg, int c, float d, float inv, float& best, int& bc) {
+  uint32_t wt[2];
+  enc16_raw(xg, inv, finite_pos(d, inv), wt);
+  const float e = sse16(xg, wt, d);
+  if (e < best || (e == best && c > bc)) { best = e; bc = c; }
 }
 
 __global__ void __launch_bounds__(256) k_mse_group(MseParams p) {
@@ -68,20 +108,21 @@ __global__ void __launch_bounds__(256) k_mse_group(MseParams p) {
   float best0 = __int_as_float(0x7F800000), best1 = best0;
   int c0 = 0, c1 = 0;
   if (gm0 > 0.0f || gm1 > 0.0f) {
+    const float xt0 = top_value(x, gm0), xt1 = top_value(x + 16, gm1);
+    // Seeds: the candidates nearest the AbsMax scale, evaluated first so that the
+    // bound below prunes from the start (any seed gives the same result).
+    const float i6 = __frcp_rn(__fmul_rn(6.0f, s_T));
+    const int sd0 = seed_code(gm0, i6), sd1 = seed_code(gm1, i6);
+    if (gm0 > 0.0f) consider(x, sd0, s_d[sd0], s_inv[sd0], best0, c0);
+    if (gm1 > 0.0f) consider(x + 16, sd1, s_d[sd1], s_inv[sd1], best1, c1);
 #pragma unroll 1
     for (int c = 1; c <= 126; ++c) {
       const float d = s_d[c], inv = s_inv[c];
       const bool ok = finite_pos(d, inv);
-      uint32_t w0[2], w1[2];
-      enc16_raw(x, inv, ok, w0);
-      enc16_raw(x + 16, inv, ok, w1);
-      const float e0 = sse16(x, w0, d), e1 = sse16(x + 16, w1, d);
-      if (e0 <= best0) { best0 = e0; c0 = c; }
-      if (e1 <= best1) { best1 = e1; c1 = c; }
+      if (gm0 > 0.0f && c != sd0 && !(top_term(xt0, d, inv, ok) > best0)) consider(x, c, d, inv, best0, c0);
+      if (gm1 > 0.0f && c != sd1 && !(top_term(xt1, d, inv, ok) > best1)) consider(x + 16, c, d, inv, best1, c1);
     }
   }
-  if (!(gm0 > 0.0f)) c0 = 0;
-  if (!(gm1 > 0.0f)) c1 = 0;
 
   uint32_t w[4];
   enc16(x, s_inv[c0], c0 != 0 && finite_pos(s_d[c0], s_inv[c0]), w);
