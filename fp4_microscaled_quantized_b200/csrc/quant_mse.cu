@@ -7,7 +7,8 @@
 // x * (1/d) and their fp32 squared error (sse16, the pairwise tree of
 // fp32((x - fp32(q d))^2)); the smallest error wins, ties to the larger code.
 // Candidates that the top element's own error term already rules out are not
-// evaluated in full (top_term); the result is that of the exhaustive scan.
+// evaluated in full (top_term), and the scan below the seed stops where that
+// term can only grow; the result is that of the exhaustive scan.
 // A group whose maximum is zero (or NaN) takes code 0 and zero codes.  With
 // the winning codes, u = E4M3(c) q is exact in fp32 and x u, u u are exact in
 // float64; the block sums both over its 8192 consecutive elements as a
@@ -72,6 +73,28 @@ __device__ __forceinline__ void consider(const float* xg, int c, float d, float 
   if (e < best || (e == best && c > bc)) { best = e; bc = c; }
 }
 
+// Candidate c above the seed: evaluated in full unless its top-element term
+// rules it out.
+__device__ __forceinline__ void probe_up(const float* xg, float xt, int c, const float* sd, const float* si,
+                                         float& best, int& bc) {
+  const float d = sd[c], inv = si[c];
+  if (!(top_term(xt, d, inv, finite_pos(d, inv)) > best)) consider(xg, c, d, inv, best, bc);
+}
+
+// Candidate c below the seed; returns whether smaller codes still need a
+// look.  Where the scale is unusable (zero codes) or fp32(6 d) <= |top|, the
+// top element's term is its clipping error (|top| - fp32(6 d))^2 (or top^2),
+// which only grows as d shrinks while the best error only falls: once such a
+// candidate is ruled out, so is every smaller one.
+__device__ __forceinline__ bool probe_down(const float* xg, float xt, int c, const float* sd, const float* si,
+                                           float& best, int& bc) {
+  const float d = sd[c], inv = si[c];
+  const bool ok = finite_pos(d, inv);
+  if (top_term(xt, d, inv, ok) > best) return ok && __fmul_rn(6.0f, d) > fabsf(xt);
+  consider(xg, c, d, inv, best, bc);
+  return true;
+}
+
 __global__ void __launch_bounds__(256) k_mse_group(MseParams p) {
   __shared__ float s_d[128], s_inv[128];
   __shared__ double s_num[8], s_den[8];
@@ -109,18 +132,25 @@ __global__ void __launch_bounds__(256) k_mse_group(MseParams p) {
   int c0 = 0, c1 = 0;
   if (gm0 > 0.0f || gm1 > 0.0f) {
     const float xt0 = top_value(x, gm0), xt1 = top_value(x + 16, gm1);
-    // Seeds: the candidates nearest the AbsMax scale, evaluated first so that the
-    // bound below prunes from the start (any seed gives the same result).
+    // Candidates are visited outward from a seed near the AbsMax scale (seed + k
+    // and seed - k at step k), so the lanes of a warp evaluate in the same steps.
     const float i6 = __frcp_rn(__fmul_rn(6.0f, s_T));
     const int sd0 = seed_code(gm0, i6), sd1 = seed_code(gm1, i6);
-    if (gm0 > 0.0f) consider(x, sd0, s_d[sd0], s_inv[sd0], best0, c0);
-    if (gm1 > 0.0f) consider(x + 16, sd1, s_d[sd1], s_inv[sd1], best1, c1);
+    const bool on0 = gm0 > 0.0f, on1 = gm1 > 0.0f;
+    if (on0) consider(x, sd0, s_d[sd0], s_inv[sd0], best0, c0);
+    if (on1) consider(x + 16, sd1, s_d[sd1], s_inv[sd1], best1, c1);
+    bool dn0 = on0, dn1 = on1;
 #pragma unroll 1
-    for (int c = 1; c <= 126; ++c) {
-      const float d = s_d[c], inv = s_inv[c];
-      const bool ok = finite_pos(d, inv);
-      if (gm0 > 0.0f && c != sd0 && !(top_term(xt0, d, inv, ok) > best0)) consider(x, c, d, inv, best0, c0);
-      if (gm1 > 0.0f && c != sd1 && !(top_term(xt1, d, inv, ok) > best1)) consider(x + 16, c, d, inv, best1, c1);
+    for (int k = 1; k <= 125; ++k) {
+      const int u0 = sd0 + k, l0 = sd0 - k, u1 = sd1 + k, l1 = sd1 - k;
+      const bool up0 = on0 && u0 <= 126, up1 = on1 && u1 <= 126;
+      dn0 = dn0 && l0 >= 1;
+      dn1 = dn1 && l1 >= 1;
+      if (!(up0 || up1 || dn0 || dn1)) break;
+      if (up0) probe_up(x, xt0, u0, s_d, s_inv, best0, c0);
+      if (up1) probe_up(x + 16, xt1, u1, s_d, s_inv, best1, c1);
+      if (dn0) dn0 = probe_down(x, xt0, l0, s_d, s_inv, best0, c0);
+      if (dn1) dn1 = probe_down(x + 16, xt1, l1, s_d, s_inv, best1, c1);
     }
   }
 
