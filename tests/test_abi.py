@@ -47,6 +47,13 @@ def test_host_helpers_without_gpu(lib):
     assert eden >= 256 + 128 * 32 * 2 + 128 * 4 * 4
     assert lib.fp4_swizzled_scale_bytes(300, 10) == 3 * 3 * 512
     assert lib.fp4_status_string(2) == b"unsupported combination"
+    lib.fp4_quantize_mse_workspace_size.restype = ctypes.c_size_t
+    lib.fp4_quantize_mse_workspace_size.argtypes = [ctypes.c_int64] * 2
+    # amax word + one float64 pair per 8192 elements, rounded up to 256 bytes
+    assert lib.fp4_quantize_mse_workspace_size(64, 256) == 256 + 256
+    assert lib.fp4_quantize_mse_workspace_size(10240, 4096) == 256 + 5120 * 16
+    assert lib.fp4_quantize_mse_workspace_size(0, 256) == 256
+    assert lib.fp4_quantize_mse_workspace_size(64, 48) == 0                 # cols not a multiple of 32
 
 
 def test_product_path_does_not_import_oracle():
