@@ -15,16 +15,18 @@ static std::atomic<unsigned long long> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add(static_cast<unsigned long long>(n)); }
 
 int num_sms() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (!v) {
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
+    v = n > 0 ? n : 148;
+    cached[dev].store(v, std::memory_order_relaxed);   // every thread computes the same value
   }
-  return cached[dev];
+  return v;
 }
 
 // Address of the status word on the current device (looked up once per device).

@@ -19,6 +19,7 @@
 // Every mbarrier wait is bounded; on timeout the kernel records
 // FP4_ERR_TIMEOUT, stops issuing work, frees its TMEM and returns.
 #include <cuda.h>
+#include <atomic>
 #include <cstdlib>
 #include <mutex>
 
@@ -972,13 +973,13 @@ template <int FMT, int OUT, int EPI>
 static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
                           cudaStream_t s) {
   auto kern = k_gemm<FMT, OUT, EPI>;
-  static bool attr_set[64] = {false};
+  static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);   // idempotent: racing threads set the same value
   }
   int64_t tiles = ((p.M + BM - 1) / BM) * ((p.N + BN - 1) / BN);
   int grid = int(tiles < num_sms() ? tiles : num_sms());
@@ -993,11 +994,12 @@ template <int FMT, int OUT, int EPI>
 static cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
                                const Params& p, cudaStream_t s) {
   auto kern = pair::k_gemm_pair<FMT, OUT, EPI>;
-  static int max_clusters[64] = {0};
+  static std::atomic<int> max_clusters[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (max_clusters[dev] == 0) {
+  int mc = max_clusters[dev].load(std::memory_order_acquire);
+  if (mc == 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pair::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -1009,10 +1011,11 @@ static cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, con
       cudaGetLastError();
       n = num_sms() / 2;
     }
-    max_clusters[dev] = n;
+    mc = n;
+    max_clusters[dev].store(mc, std::memory_order_release);   // idempotent: racing threads store the same value
   }
   const int64_t tiles = ((p.M + 255) / 256) * ((p.N + BN - 1) / BN);
-  const int64_t pairs = tiles < max_clusters[dev] ? tiles : max_clusters[dev];
+  const int64_t pairs = tiles < mc ? tiles : mc;
   kern<<<unsigned(2 * pairs), pair::PTHREADS, pair::SMEM_BYTES, s>>>(ma, mb, md, p);
   count_launch();
   return cudaGetLastError();

@@ -1,6 +1,8 @@
 // Host-side launch of the quantiser kernels for one loader (instantiated once
 // per loader in quant_ld*.cu so the four compile in parallel).
 #pragma once
+#include <atomic>
+
 #include "quant_core32.cuh"
 
 namespace fp4 {
@@ -16,17 +18,19 @@ int num_sms();
 // and then runs alone at the end.
 template <bool WIDE, int LOAD, int FMT, int RND, int HAD>
 int resident_blocks() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (!cached[dev]) {
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (!v) {
     int n = 0;
     cudaError_t e = WIDE ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row32<LOAD, FMT, RND, HAD>, 256, 0)
                          : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row<LOAD, FMT, RND, HAD>, 256, 0);
-    cached[dev] = (e == cudaSuccess && n >= 1) ? n : 1;
+    v = (e == cudaSuccess && n >= 1) ? n : 1;
+    cached[dev].store(v, std::memory_order_relaxed);   // every thread computes the same value
   }
-  return cached[dev];
+  return v;
 }
 
 template <int LOAD, int FMT, int RND, int HAD>
