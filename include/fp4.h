@@ -164,7 +164,8 @@ int fp4_transpose_square16(const fp4_qtensor *in, fp4_qtensor *out, fp4_stream_t
  * Launches 2 + 2 * iters kernels (plus one when the swizzled scales need
  * padding).  A non-finite input sets FP4_ERR_NONFINITE_INPUT on the device.
  * Errors: FP4_ERR_INVALID_ARG (shape, iters, null pointers),
- * FP4_ERR_ALIGNMENT, FP4_ERR_WORKSPACE. */
+ * FP4_ERR_ALIGNMENT, FP4_ERR_WORKSPACE, FP4_ERR_CUDA (a launch failed).
+ * fp4_quantize_mse_workspace_size returns 0 for an invalid shape. */
 size_t fp4_quantize_mse_workspace_size(int64_t rows, int64_t cols);
 int fp4_quantize_mse(const void *x_dev, int64_t rows, int64_t cols, int32_t iters,
                      fp4_qtensor *out, void *ws_dev, size_t ws_bytes, fp4_stream_t stream);
