@@ -471,6 +471,20 @@ def oracle_sample(n_rows, n_out, seed=0):
     return flops, dt
 
 
+def host_cpu():
+    """The host's CPU model and logical core count, recorded beside the oracle's timing."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return "%s, %d logical cores" % (model, os.cpu_count() or 0)
+
+
 def cpu_baseline(target_s=15.0):
     # calibrate on a small sample, then run one sized for about target_s
     f0, t0 = oracle_sample(128, 256)
@@ -478,7 +492,7 @@ def cpu_baseline(target_s=15.0):
     f1, t1 = oracle_sample(128, n_out)
     return {"value": f1 / t1 / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": "QKV layer, 128 tokens x %d output features x K=4096, Quartet II fwd+bwd "
-                      "(quantisers + fp64 GEMMs), %.1f s" % (n_out, t1)}
+                      "(quantisers + fp64 GEMMs), %.1f s" % (n_out, t1), "host": host_cpu()}
 
 
 def reference_arm(args, world, rank):
@@ -501,7 +515,8 @@ def reference_arm(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantisers, f64 GEMM",
         "data": "synthetic", "config": config_dict(M_TOKENS),
-        "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                         "host": host_cpu()},
         "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
 
 
