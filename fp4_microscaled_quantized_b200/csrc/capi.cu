@@ -281,9 +281,17 @@ size_t fp4_swizzled_scale_bytes(int64_t rows, int64_t n_groups) {
   return size_t((rows + 127) / 128) * size_t((n_groups + 3) / 4) * 512;
 }
 
-int fp4_quantize(const void* x, int64_t in_rows, int64_t in_cols, int32_t transpose, int32_t fmt,
-                 int32_t rounding, int32_t group, fp4_had had, uint64_t seed, uint32_t tensor_tag,
-                 fp4_qtensor* out, void* ws, size_t ws_bytes, fp4_stream_t stream) {
+}  // extern "C"
+
+namespace fp4 {
+// Every argument check of fp4_quantize before its workspace check, in the
+// same order (fp4_quantize_noalloc runs them before its scratch-size check so
+// both entry points return the same status for the same arguments).  Sets
+// out's shape fields; *empty is set for a tensor with no elements (valid,
+// nothing to launch).
+static int quantize_args(const void* x, int64_t in_rows, int64_t in_cols, int32_t transpose, int32_t fmt,
+                         int32_t rounding, int32_t group, fp4_had had, fp4_qtensor* out, bool* empty) {
+  *empty = false;
   if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
   if (rounding < FP4_RTN || rounding > FP4_RTN_SQUARE16) return FP4_ERR_INVALID_ARG;
   const int g = fmt == FP4_NVFP4 ? 16 : 32;
@@ -300,11 +308,27 @@ int fp4_quantize(const void* x, int64_t in_rows, int64_t in_cols, int32_t transp
   if (transpose && (in_cols % 8)) return FP4_ERR_ALIGNMENT;
   if (transpose && had.block > 128) return FP4_ERR_UNSUPPORTED;   // longer than the transposed tile
   out->rows = rows; out->cols = cols; out->fmt = fmt;
-  if (rows == 0 || cols == 0) return FP4_OK;   // empty tensor: nothing to launch
+  if (rows == 0 || cols == 0) {   // empty tensor: nothing to launch
+    *empty = true;
+    return FP4_OK;
+  }
   int st = check_out(out);
   if (st) return st;
   if (!x) return FP4_ERR_INVALID_ARG;
   if (!aligned(x, 16)) return FP4_ERR_ALIGNMENT;
+  return FP4_OK;
+}
+}  // namespace fp4
+
+extern "C" {
+
+int fp4_quantize(const void* x, int64_t in_rows, int64_t in_cols, int32_t transpose, int32_t fmt,
+                 int32_t rounding, int32_t group, fp4_had had, uint64_t seed, uint32_t tensor_tag,
+                 fp4_qtensor* out, void* ws, size_t ws_bytes, fp4_stream_t stream) {
+  bool empty = false;
+  const int st = quantize_args(x, in_rows, in_cols, transpose, fmt, rounding, group, had, out, &empty);
+  if (st || empty) return st;
+  const int64_t rows = out->rows, cols = out->cols;
   QParams p{};
   p.x = x; p.in_rows = in_rows; p.in_cols = in_cols; p.rows = rows; p.cols = cols;
   p.codes = out->codes; p.scales = out->scales; p.swz = out->scales_swz; p.mask = out->mask;
@@ -546,8 +570,12 @@ static void* noalloc_scratch_ptr() {
 extern "C" int fp4_quantize_noalloc(const void* x, int64_t in_rows, int64_t in_cols, int32_t transpose,
                                     int32_t fmt, int32_t rounding, int32_t group, fp4_had had, uint64_t seed,
                                     uint32_t tensor_tag, fp4_qtensor* out, fp4_stream_t stream) {
-  if (in_rows < 0 || in_cols < 0 || (transpose != 0 && transpose != 1)) return FP4_ERR_INVALID_ARG;
-  const int64_t rows = transpose ? in_cols : in_rows, cols = transpose ? in_rows : in_cols;
+  // fp4_quantize's own argument checks first, so both calls give the same
+  // status for the same arguments; then the size of the scratch.
+  bool empty = false;
+  const int st = quantize_args(x, in_rows, in_cols, transpose, fmt, rounding, group, had, out, &empty);
+  if (st || empty) return st;
+  const int64_t rows = out->rows, cols = out->cols;
   const size_t need = fp4_quantize_workspace_size(rows, cols, fmt, rounding, had.block);
   if (need > FP4_NOALLOC_SCRATCH_BYTES) return FP4_ERR_WORKSPACE;   // tensor too large for the array
   void* ws = nullptr;

@@ -215,8 +215,11 @@ int fp4_quantize(const void *x_dev, int64_t in_rows, int64_t in_cols,
  *  - Limit: a quantised tensor whose fp4_quantize_workspace_size exceeds
  *    FP4_NOALLOC_SCRATCH_BYTES (4 MiB) returns FP4_ERR_WORKSPACE and launches
  *    nothing.  That is about 26.8 million elements for MS-EDEN with 128-blocks
- *    (16.7 million with 32-blocks, 11.1 million with 16-blocks); the other
- *    NVFP4 modes (256 bytes) and all MXFP4 modes (none) fit at any size.
+ *    (16.7 million with 32-blocks, 11.1 million with 16-blocks) and about 268
+ *    million for FP4_RTN_SQUARE16 (256 + rows * cols / 64 bytes: one fp32
+ *    maximum per 16 x 16 block); the other NVFP4 modes (256 bytes) and all
+ *    MXFP4 modes (none) fit at any size.  An invalid argument returns the
+ *    same status as fp4_quantize, whatever the size.
  *  - All calls share the one array and it keeps the last call's contents; the
  *    part that must start at zero (the amax word) is cleared on `stream`
  *    inside the call.  Two calls whose work overlaps on the GPU (different

@@ -162,3 +162,45 @@ def test_recipe_validation(lib):
     ctx = api.fp4_ctx()
     assert lib.fp4_linear_fwd(FAKE, FAKE, 256, 512, 1024, ctypes.byref(r), 0, FAKE, ctypes.byref(ctx),
                               FAKE, 1 << 30, None) == INVALID
+
+
+def _noalloc(lib, x, in_rows, in_cols, fmt, rnd, group, had=0, transpose=0, out=None):
+    f = lib.fp4_quantize_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_int32, ctypes.c_int32, api.fp4_had, ctypes.c_uint64, ctypes.c_uint32,
+                  ctypes.POINTER(api.fp4_qtensor), ctypes.c_void_p]
+    out = out if out is not None else fake_out()
+    return f(x, in_rows, in_cols, transpose, fmt, rnd, group, api.fp4_had(had, 0, 0), 0, 0, ctypes.byref(out), None)
+
+
+@pytest.mark.parametrize("fmt,rnd,group,had,shape,transpose,want", [
+    # a tensor far larger than the 4 MiB scratch: the argument errors still come first
+    (1, 4, 16, 8, (8192, 8192), 0, UNSUPPORTED),            # MS-EDEN with block 8
+    (1, 4, 16, 48, (8192, 8160), 0, UNSUPPORTED),           # MS-EDEN with block 48
+    (1, 4, 16, 128, (8192, 8200), 0, INVALID),              # inner dim not a multiple of 128
+    (1, 0, 32, 0, (8192, 8192), 0, UNSUPPORTED),            # wrong group for NVFP4
+    (1, 4, 16, 128, (8192, 8196), 1, ALIGNMENT),            # transposed: input rows of 8196 elements
+    # valid arguments beyond the scratch: the size check
+    (1, 4, 16, 128, (8192, 8192), 0, WORKSPACE),
+    (1, 5, 16, 0, (32768, 16384), 0, WORKSPACE),            # square blocks: 256 + rows * cols / 64 bytes
+])
+def test_quantize_noalloc_status_matches_quantize(lib, fmt, rnd, group, had, shape, transpose, want):
+    """fp4_quantize_noalloc returns fp4_quantize's status for an invalid
+    argument, whatever the tensor's size; only valid arguments reach its own
+    scratch-size check (all before any CUDA call)."""
+    assert _noalloc(lib, FAKE, shape[0], shape[1], fmt, rnd, group, had, transpose) == want
+    if want != WORKSPACE:
+        assert quantize(lib, FAKE, shape[0], shape[1], fmt, rnd, group, had, transpose) == want
+
+
+def test_quantize_noalloc_square_block_limit(lib):
+    """The square-block mode keeps one fp32 maximum per 16 x 16 block in the
+    scratch: 256 + rows * cols / 64 bytes, so 4 MiB holds about 268 million
+    elements."""
+    need = lib.fp4_quantize_workspace_size(16384, 16352, 1, 5, 0)
+    assert need == 256 + 16384 * 16352 // 64
+    assert need <= 4 << 20
+    assert lib.fp4_quantize_workspace_size(16384, 16384, 1, 5, 0) > 4 << 20
+    empty = api.fp4_qtensor()
+    assert _noalloc(lib, None, 0, 64, 1, 5, 16, out=empty) == OK

@@ -35,10 +35,14 @@ def _same(a, b):
     (1, 4, 128, True),
     (1, 2, 0, False),       # NVFP4 Four-Over-Six: amax word in the scratch
     (0, 3, 32, False),      # MXFP4 SR: no scratch at all
+    (1, 5, 0, False),       # NVFP4 16 x 16 square blocks: one maximum per block in the scratch
+    (1, 5, 0, True),
 ])
 def test_noalloc_matches_regular_quantize_twice(cuda_lib, fmt, rnd, had, transpose):
     first = _dev(syn.student_t((1024, 2048), seed=21, unit_rms=True))
-    second = _dev(syn.outlier_elements((1024, 2048), seed=22))      # different data, smaller amax
+    # different data with a far smaller amax and block maxima, so anything
+    # left in the shared scratch by the first call would change the second
+    second = _dev(syn.gaussian((1024, 2048), 0.02, seed=22))
     for k, x in enumerate((first, second)):
         ref = cuda_lib.quantize(x, fmt, rnd, had, randomized=True, seed=5 + k, tensor_tag=3,
                                 transpose=transpose)
