@@ -83,6 +83,9 @@ QCASES = {
     "W_four_over_six": ("w", qn.NVFP4, qn.FOUR_OVER_SIX, 0, False, 0, ln.TAG_W),
     # the quantiser sweep's 2^28-element point (rows of 4096, N(0,1) + 0.1% x 50)
     "sweep_2e28_nvfp4_sr_h32": ("sweep", qn.NVFP4, qn.SR, 32, False, 0, 9),
+    "sweep_2e28_nvfp4_eden_h128_t": ("sweep", qn.NVFP4, qn.MS_EDEN, 128, True, 1, 10),
+    "sweep_2e28_nvfp4_fos_h0": ("sweep", qn.NVFP4, qn.FOUR_OVER_SIX, 0, False, 0, 11),
+    "sweep_2e28_mxfp4_quest_h32": ("sweep", qn.MXFP4, qn.QUEST, 32, False, 0, 12),
 }
 
 
@@ -102,11 +105,12 @@ def test_quantizer_full_size(cuda_lib, qkv_data, request, name):
     bits = request.getfixturevalue("sweep_data") if src == "sweep" else \
         {"dy": qkv_data["dY"], "x": qkv_data["X"], "w": qkv_data["W"]}[src]
     seed = 1234
-    g = cuda_lib.quantize(dev(bits), fmt, rnd, had, randomized=had > 0, seed=seed, sign_tag=sign_tag,
+    rand = had > 0 and rnd in (qn.SR, qn.MS_EDEN)      # the backward modes rotate randomly, the others do not
+    g = cuda_lib.quantize(dev(bits), fmt, rnd, had, randomized=rand, seed=seed, sign_tag=sign_tag,
                           tensor_tag=tag, transpose=transpose)
     n_out = bits.shape[1] if transpose else bits.shape[0]
     rows = sample(n_out, seed=len(name))
-    o = qn.quantize_rows(f32(bits), rows, fmt, rnd, had, randomized=had > 0, seed=seed, sign_tag=sign_tag,
+    o = qn.quantize_rows(f32(bits), rows, fmt, rnd, had, randomized=rand, seed=seed, sign_tag=sign_tag,
                          tensor_tag=tag, transpose=transpose)
     check_rows(g, o, rows)
     assert cuda_lib.get_last_error() == 0
@@ -223,4 +227,43 @@ def test_linear_quartet_full_size(cuda_lib):
     dw, bw = gm.gemm_ref(e_t, x_t)
     dw_ref, dwb = gm.quartet_epilogue_ref(dw, bw, ~mask_w, rec.fwd_had)
     check_block(dW, nb, kb, dw_ref, dwb)
+    assert cuda_lib.get_last_error() == 0
+
+
+def test_linear_layer_set_gate_up_full_size(cuda_lib):
+    """The layer set's gate/up layer at M = 16384 (K = 4096, N = 28672, data
+    seed 5 as in the bench) through fp4_linear_fwd / fp4_linear_bwd: the two
+    longest accumulations the bench times, dX = E W (inner N = 28672) and
+    dW = E^T X (inner M = 16384), on sampled rows x columns against fp64
+    products of the oracle's own operands (its whole-tensor Four-Over-Six of
+    X and W, de-quantised, and its MS-EDEN of the sampled rows with the
+    whole transformed tensors' amax)."""
+    M, K, N, step = 16384, 4096, 28672, 3
+    d = syn.linear_quartet2(M, N, K, seed=5)
+    r = cuda_lib.recipe(cuda_lib.RECIPE_QUARTET2)
+    Y, ctx = cuda_lib.linear_fwd(dev(d["X"]), dev(d["W"]), r, seed=0)
+    dX, dW = cuda_lib.linear_bwd(dev(d["dY"]), ctx, step)
+    torch.cuda.synchronize()
+    X, W, dY = f32(d["X"]), f32(d["W"]), f32(d["dY"])
+    del d
+    rm, rn, rk = sample(M, k=12, seed=31), sample(N, k=12, seed=32), sample(K, k=12, seed=33)
+    oxq, owq = qn.nvfp4_four_over_six(X), qn.nvfp4_four_over_six(W)
+    check_rows(ctx.xq, qn.QTensor(oxq.codes[rm], oxq.scales[rm], oxq.tensor_scale, oxq.fmt), rm)
+    y_ref, yb = gm.gemm_ref(qn.QTensor(oxq.codes[rm], oxq.scales[rm], oxq.tensor_scale, oxq.fmt),
+                            qn.QTensor(owq.codes[rn], owq.scales[rn], owq.tensor_scale, owq.fmt))
+    check_block(Y, rm, rn, y_ref, yb)
+    deq_x, deq_w = qn.dequant_f32(oxq), qn.dequant_f32(owq)
+    del oxq, owq, X, W
+    kw = dict(randomized=True, seed=step)
+    e_row = qn.quantize_rows(dY, rm, qn.NVFP4, qn.MS_EDEN, 128, sign_tag=ln.GEMM_DX, tensor_tag=ln.TAG_E_ROW, **kw)
+    w_t = qn.quantize_rows(deq_w, rk, qn.NVFP4, qn.MS_EDEN, 128, sign_tag=ln.GEMM_DX, tensor_tag=ln.TAG_W_T,
+                           transpose=True, **kw)
+    dx_ref, dxb = gm.gemm_ref(e_row, w_t)
+    check_block(dX, rm, rk, dx_ref, dxb)
+    e_t = qn.quantize_rows(dY, rn, qn.NVFP4, qn.MS_EDEN, 128, sign_tag=ln.GEMM_DW, tensor_tag=ln.TAG_E_T,
+                           transpose=True, **kw)
+    x_t = qn.quantize_rows(deq_x, rk, qn.NVFP4, qn.MS_EDEN, 128, sign_tag=ln.GEMM_DW, tensor_tag=ln.TAG_X_T,
+                           transpose=True, **kw)
+    dw_ref, dwb = gm.gemm_ref(e_t, x_t)
+    check_block(dW, rn, rk, dw_ref, dwb)
     assert cuda_lib.get_last_error() == 0
