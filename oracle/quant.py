@@ -652,3 +652,80 @@ def swizzle_scales(scales):
     off = ((r // 128) * nkb + k // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + k % 4
     out[off.reshape(-1)] = scales.reshape(-1)
     return out
+
+
+# ----------------------------------------------------- MXFP4 scale fit ----
+@dataclass
+class FitTensor:
+    """MXFP4 with fitted fractional-exponent scales (MXFP4-dagger): E2M1
+    codes, one 8-bit level q per 32-element group and the tensor's table of
+    the 256 scale values 2^(alpha q + beta)."""
+    codes: np.ndarray          # (rows, cols) uint8
+    q: np.ndarray              # (rows, cols // 32) uint8
+    table: np.ndarray          # (256,) float32
+    thresholds: np.ndarray     # (255,) float32, level k -> k + 1 boundary
+    l_min: float
+    alpha: float
+
+
+def mxfp4_fit_levels(s_min, s_max):
+    """Bridging-the-Gap page, "MXFP Scale Fitting" (Appendix H, the
+    MXFP4-dagger remap): with L = log2 of the smallest and largest group
+    scale of the tensor, level q in [0, 255] stands for the scale
+    2^(alpha q + L_min), alpha = (L_max - L_min) / 255 -- a fractional
+    exponent step (READING: the printed formula is garbled, it multiplies the
+    level by L_max - L_min; the page's own summary s = 2^(alpha q + beta) with
+    alpha in (0, 1) fixes the 1/255).  Level k and k + 1 meet where the
+    log-scale crosses alpha (k + 0.5), the page's round().  Returns the fp32
+    table of the 256 scales, the 255 fp32 boundaries, L_min and alpha; every
+    exponent is computed in fp64 and rounded once to fp32."""
+    l_min = float(np.log2(np.float64(s_min)))
+    l_max = float(np.log2(np.float64(s_max)))
+    alpha = (l_max - l_min) / 255.0
+    q = np.arange(256, dtype=np.float64)
+    table = np.exp2(l_min + alpha * q).astype(F32)
+    thr = np.exp2(l_min + alpha * (q[:255] + 0.5)).astype(F32)
+    return table, thr, l_min, alpha
+
+
+def mxfp4_fit(x):
+    """MXFP4-dagger quantisation of an (already transformed) fp32 tensor,
+    RTN elements.  READINGS: the group scale before fitting is the AbsMax
+    scale s = fp32(gmax / 6) (the modified formula drops the 4/3 bias of the
+    original rule); L_min and L_max come from the groups with s > 0; a
+    group's level is the number of boundaries t_k with s >= t_k (the
+    round() of the page, ties up); the elements are RTN_E2M1(x * fp32(1/d))
+    with d = table[q], saturating at 6, as the other RTN rules here; a group
+    with s = 0, or whose reciprocal scale is not finite, encodes as zeros
+    with level 0; a tensor with no s > 0 gets the table of s = 1; when every
+    s > 0 is equal, alpha = 0, all levels and boundaries equal s and the
+    count gives level 255.
+    (The E8M0 block scaling of the tensor cores cannot apply these scales:
+    they are not powers of two.)"""
+    x = np.asarray(x, dtype=F32)
+    rows, cols = x.shape
+    xg = _groups(x, 32)
+    s = (_group_max(xg) / F32(6.0)).astype(F32)
+    pos = s > 0
+    if pos.any():
+        table, thr, l_min, alpha = mxfp4_fit_levels(s[pos].min(), s[pos].max())
+    else:
+        table, thr, l_min, alpha = mxfp4_fit_levels(F32(1.0), F32(1.0))
+    q = (s[..., None] >= thr).sum(axis=-1).astype(np.int64)
+    q = np.where(pos, q, 0)
+    d = table[q]
+    with np.errstate(divide="ignore", over="ignore"):
+        inv = (F32(1.0) / d).astype(F32)
+    ok = pos & np.isfinite(inv)
+    v = (xg * np.where(ok, inv, F32(0.0))[..., None]).astype(F32)
+    codes = fm.rtn_e2m1(v).reshape(rows, cols)
+    return FitTensor(codes, q.astype(np.uint8), table, thr, l_min, alpha)
+
+
+def mxfp4_fit_dequant(ft):
+    """fp32(code * table[q]) per element (q * d is exact: one significant
+    bit pair times an fp32 scale)."""
+    rows, cols = ft.codes.shape
+    q = fm.decode_e2m1(ft.codes).reshape(rows, cols // 32, 32)
+    d = ft.table[ft.q.astype(np.int64)]
+    return (q * d[..., None]).astype(F32).reshape(rows, cols)
