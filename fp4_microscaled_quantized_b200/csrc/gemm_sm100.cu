@@ -205,6 +205,15 @@ __device__ __forceinline__ uint32_t idesc(int fmt, int n, int m, uint32_t sfa_id
   return d;
 }
 
+// The MMAs of one full k-tile (NK of K = 64), unrolled: the operand
+// descriptors advance by 32 bytes (2 in their 16-byte address field) per MMA,
+// the scale-factor TMEM addresses by one atom (4 columns of A, 8 of B; MXFP4
+// takes two MMAs per atom, bytes 0-1 then 2-3), and only the first MMA of a
+// tile's first k-tile overwrites the accumulator.
+template <int FMT, int NK, bool PAIR = false>
+__device__ __forceinline__ void mma_ktile(uint32_t acc, uint64_t ad, uint64_t bd, uint32_t sfbase, uint32_t idesc0,
+                                          bool accumulate);
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
   asm volatile(
@@ -317,15 +326,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
         const int n_mma = kel / 64;
-        const uint32_t a_base = smem_u32(sA + s * A_BYTES), b_base = smem_u32(sB + s * B_BYTES);
+        const uint64_t ad = desc_sw128(smem_u32(sA + s * A_BYTES)), bd = desc_sw128(smem_u32(sB + s * B_BYTES));
         const uint32_t sfbase = tmem + SF_COL + SF_BUF_COLS * uint32_t(buf);
-        for (int kk = 0; kk < n_mma; ++kk) {
-          const int atom = FMT == 1 ? kk : kk / 2;
-          const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
-          const uint32_t sfa = (sfbase + 4 * atom) | (sf_id << 30);
-          const uint32_t sfb = (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30);
-          tc_mma<FMT>(tmem + ACC_COL, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
-                      idesc(FMT, BN, BM, sf_id, sf_id), sfa, sfb, (kt > 0 || kk > 0) ? 1u : 0u);
+        if (n_mma == BK / 64) {
+          mma_ktile<FMT, BK / 64>(tmem + ACC_COL, ad, bd, sfbase, idesc(FMT, BN, BM, 0, 0), kt > 0);
+        } else {                                          // the last, partial k-tile
+          for (int kk = 0; kk < n_mma; ++kk) {
+            const int atom = FMT == 1 ? kk : kk / 2;
+            const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
+            tc_mma<FMT>(tmem + ACC_COL, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk),
+                        idesc(FMT, BN, BM, sf_id, sf_id), (sfbase + 4 * atom) | (sf_id << 30),
+                        (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30), (kt > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         tc_commit(&empty[s]);
         tc_commit(&sf_empty[buf]);
@@ -610,6 +622,25 @@ __device__ __forceinline__ void mma_pair(uint32_t d, uint64_t a, uint64_t b, uin
   }
 }
 
+}  // namespace pair
+
+template <int FMT, int NK, bool PAIR>
+__device__ __forceinline__ void mma_ktile(uint32_t acc, uint64_t ad, uint64_t bd, uint32_t sfbase, uint32_t idesc0,
+                                          bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < NK; ++kk) {
+    const int atom = FMT == 1 ? kk : kk / 2;
+    const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
+    const uint32_t id = idesc0 | (sf_id << 4) | (sf_id << 29);
+    const uint32_t sfa = (sfbase + 4 * atom) | (sf_id << 30), sfb = (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30);
+    const uint32_t c = (kk > 0 || accumulate) ? 1u : 0u;
+    if (PAIR) pair::mma_pair<FMT>(acc, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), id, sfa, sfb, c);
+    else tc_mma<FMT>(acc, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), id, sfa, sfb, c);
+  }
+}
+
+namespace pair {
+
 // Pair tile order.  raster > 0: groups of `raster` 256-row blocks sweep all
 // 256-column blocks (each B tile is fetched once per group and shared by the
 // group's tiles of one wave); raster < 0: groups of -raster column blocks
@@ -742,15 +773,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         tc_fence_after();
         const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
         const int n_mma = kel / 64;
-        const uint32_t a_base = smem_u32(sA + s * A_BYTES), b_base = smem_u32(sB + s * B_BYTES);
+        const uint64_t ad = desc_sw128(smem_u32(sA + s * A_BYTES)), bd = desc_sw128(smem_u32(sB + s * B_BYTES));
         const uint32_t sfbase = tmem + SF_COL + SF_BUF_COLS * uint32_t(buf);
-        for (int kk = 0; kk < n_mma; ++kk) {
-          const int atom = FMT == 1 ? kk : kk / 2;
-          const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
-          const uint32_t sfa = (sfbase + 4 * atom) | (sf_id << 30);
-          const uint32_t sfb = (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30);
-          mma_pair<FMT>(tmem + ACC_COL, desc_sw128(a_base + kk * 32), desc_sw128(b_base + kk * 32),
-                        idesc(FMT, BN, 256, sf_id, sf_id), sfa, sfb, (kt > 0 || kk > 0) ? 1u : 0u);
+        if (n_mma == BK / 64) {
+          mma_ktile<FMT, BK / 64, true>(tmem + ACC_COL, ad, bd, sfbase, idesc(FMT, BN, 256, 0, 0), kt > 0);
+        } else {                                          // the last, partial k-tile
+          for (int kk = 0; kk < n_mma; ++kk) {
+            const int atom = FMT == 1 ? kk : kk / 2;
+            const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
+            mma_pair<FMT>(tmem + ACC_COL, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc(FMT, BN, 256, sf_id, sf_id),
+                          (sfbase + 4 * atom) | (sf_id << 30), (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30),
+                          (kt > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         issued = true;
         commit_both(&empty[s]);
