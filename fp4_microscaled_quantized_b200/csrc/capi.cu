@@ -224,6 +224,7 @@ static int run_quant(int load, int fmt, int rnd, int had, QParams& p, void* ws, 
       case LD_ROW: return launch_quant<LD_ROW>(fmt, r, had, p, s);
       case LD_TRANS: return launch_quant<LD_TRANS>(fmt, r, had, p, s);
       case LD_ROW_FP4: return launch_quant<LD_ROW_FP4>(fmt, r, had, p, s);
+      case LD_ROW_F32: return launch_quant<LD_ROW_F32>(fmt, r, had, p, s);
       default: return launch_quant<LD_TRANS_FP4>(fmt, r, had, p, s);
     }
   };
@@ -306,7 +307,6 @@ static int quantize_args(const void* x, int64_t in_rows, int64_t in_cols, int32_
   const int64_t chunk = had.block > g ? had.block : g;
   if (cols % chunk) return FP4_ERR_INVALID_ARG;
   if (transpose && (in_cols % 8)) return FP4_ERR_ALIGNMENT;
-  if (transpose && had.block > 128) return FP4_ERR_UNSUPPORTED;   // longer than the transposed tile
   out->rows = rows; out->cols = cols; out->fmt = fmt;
   if (rows == 0 || cols == 0) {   // empty tensor: nothing to launch
     *empty = true;
@@ -338,6 +338,29 @@ int fp4_quantize(const void* x, int64_t in_rows, int64_t in_cols, int32_t transp
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
+int fp4_quantize_f32(const float* y, int64_t rows, int64_t cols, int32_t fmt, int32_t rounding, int32_t group,
+                     uint64_t seed, uint32_t tensor_tag, fp4_qtensor* out, void* ws, size_t ws_bytes,
+                     fp4_stream_t stream) {
+  if (fmt != FP4_MXFP4 && fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+  if (rounding < FP4_RTN || rounding > FP4_RTN_SQUARE16) return FP4_ERR_INVALID_ARG;
+  if (group != (fmt == FP4_NVFP4 ? 16 : 32)) return FP4_ERR_UNSUPPORTED;
+  // MS-EDEN needs its own rotation; square blocks read bf16 block maxima
+  if (rounding == FP4_MS_EDEN || rounding == FP4_RTN_SQUARE16 || !combo_supported(fmt, rounding, 0))
+    return FP4_ERR_UNSUPPORTED;
+  if (rows < 0 || cols < 0 || cols % 32 || !out) return FP4_ERR_INVALID_ARG;
+  out->rows = rows; out->cols = cols; out->fmt = fmt;
+  if (rows == 0 || cols == 0) return FP4_OK;
+  int st = check_out(out);
+  if (st) return st;
+  if (!y) return FP4_ERR_INVALID_ARG;
+  if (!aligned(y, 16)) return FP4_ERR_ALIGNMENT;
+  QParams p{};
+  p.x = y; p.in_rows = rows; p.in_cols = cols; p.rows = rows; p.cols = cols;
+  p.codes = out->codes; p.scales = out->scales; p.swz = out->scales_swz; p.mask = out->mask;
+  p.ts = out->tensor_scale; p.seed = seed; p.tensor_tag = tensor_tag;
+  return run_quant(LD_ROW_F32, fmt, rounding, 0, p, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int fp4_requantize(const fp4_qtensor* in, int32_t transpose, int32_t rounding, fp4_had had,
                    uint64_t seed, uint32_t tensor_tag, fp4_qtensor* out, void* ws, size_t ws_bytes,
                    fp4_stream_t stream) {
@@ -355,7 +378,6 @@ int fp4_requantize(const fp4_qtensor* in, int32_t transpose, int32_t rounding, f
   const int64_t chunk = had.block > g ? had.block : g;
   if (cols % chunk) return FP4_ERR_INVALID_ARG;
   if (transpose && (in->cols % 16)) return FP4_ERR_ALIGNMENT;
-  if (transpose && had.block > 128) return FP4_ERR_UNSUPPORTED;   // longer than the transposed tile
   out->rows = rows; out->cols = cols; out->fmt = fmt;
   if (rows == 0 || cols == 0) return FP4_OK;
   int st = check_out(out);

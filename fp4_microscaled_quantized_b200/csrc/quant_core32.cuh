@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
   const uint32_t sw = lane_signs<HAD>(sh, p, 32 * (lane & 7));
   uint32_t sm[LOAD == LD_ROW ? 16 : 4];
   if (LOAD == LD_ROW) sign_masks_bf16(sw, sm);
-  else sign_masks_fp4(sw, sm);
+  else if (LOAD == LD_ROW_FP4) sign_masks_fp4(sw, sm);
   // Row and column task of t = base + lane, advanced by the grid stride
   // without a division per task.
   const int64_t base0 = int64_t(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
@@ -548,6 +548,13 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
         v[i].x ^= sm[4 * i]; v[i].y ^= sm[4 * i + 1]; v[i].z ^= sm[4 * i + 2]; v[i].w ^= sm[4 * i + 3];
         bf16x8_to_f32(v[i], x + 8 * i);
       }
+    } else if (LOAD == LD_ROW_F32) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.x) + orow * p.cols + ocol);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = active ? __ldg(src + i) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        x[4 * i] = v.x; x[4 * i + 1] = v.y; x[4 * i + 2] = v.z; x[4 * i + 3] = v.w;
+      }
     } else {
       uint4 cw = make_uint4(0, 0, 0, 0);
       uint32_t s0 = 0, s1 = 0;
@@ -570,22 +577,33 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
   if (RND == R_AMAX || RND == R_EDEN) block_max_atomic(acc, sh, p.amax_bits, p.status);
 }
 
-// Transposed, 32 elements per lane: the 128 x 64 input tile is staged as fp32
-// with a 4-float skew every 32 columns, so the 16-byte reads of four lanes on
-// one 128-element output row hit distinct banks.
-constexpr int T32_PITCH = 144;
+// Transposed, 32 elements per lane: an input tile of T32Tile::ROWS rows (the
+// output rows' length covered by one block: 128, or 256 for 256-element
+// rotation blocks) x T32Tile::COLS columns (8192 elements) is staged as fp32
+// with a 4-float skew every 32 columns, so the 16-byte reads of the lanes on
+// one output row hit distinct banks.
+template <int HAD>
+struct T32Tile {
+  static constexpr int ROWS = HAD > 128 ? 256 : 128;   // input rows = output columns per block
+  static constexpr int COLS = 8192 / ROWS;               // input columns = output rows per block
+  static constexpr int PITCH = ROWS + ROWS / 8;          // + 4 floats per 32
+  static constexpr int LPR = ROWS / 32;                  // lanes per output row
+};
 __device__ __forceinline__ int t32_col(int c) { return c + 4 * (c >> 5); }
 
 template <int LOAD, int FMT, int RND, int HAD>
 __global__ void __launch_bounds__(256, quant_trans_min_blocks<RND>()) k_quant_trans32(QParams p) {
+  using TT = T32Tile<HAD>;
   __shared__ Shared sh;
-  __shared__ __align__(16) float tile[TR_IN_COLS][T32_PITCH];
+  __shared__ __align__(16) float tile[TT::COLS][TT::PITCH];
   load_signs<HAD>(sh, p);
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t r0 = int64_t(blockIdx.x) * TR_IN_ROWS, c0 = int64_t(blockIdx.y) * TR_IN_COLS;
+  const int64_t r0 = int64_t(blockIdx.x) * TT::ROWS, c0 = int64_t(blockIdx.y) * TT::COLS;
   const int64_t R = p.in_rows, C = p.in_cols;
   {
-    const int rh = w >> 2, cb = w & 3;
+    // warp w loads input rows 64 rh + 2 lane (+1) and 16 columns 16 cb ..
+    constexpr int NCB = TT::COLS / 16;
+    const int rh = w / NCB, cb = w % NCB;
     const int rl = 64 * rh + 2 * lane;
     const int64_t cc = c0 + 16 * cb;
     float va[16], vb[16];
@@ -642,7 +660,7 @@ __global__ void __launch_bounds__(256, quant_trans_min_blocks<RND>()) k_quant_tr
   const uint32_t amax_in = (FMT == FMT_NV && RND != R_EDEN && RND != R_AMAX) ? *p.amax_bits : 0u;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) write_tensor_scale<FMT, RND>(p, amax_in);
   const QuantConsts qc = quant_consts<FMT, RND>(amax_in);
-  const int orl = threadIdx.x >> 2, seg = threadIdx.x & 3;
+  const int orl = threadIdx.x / TT::LPR, seg = threadIdx.x % TT::LPR;
   const int64_t orow = c0 + orl, ocol = r0 + 32 * seg;
   const bool active = orow < C && ocol < R;
   float x[32];

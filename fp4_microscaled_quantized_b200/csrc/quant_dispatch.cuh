@@ -25,8 +25,9 @@ int resident_blocks() {
   int v = cached[dev].load(std::memory_order_relaxed);
   if (!v) {
     int n = 0;
-    cudaError_t e = WIDE ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row32<LOAD, FMT, RND, HAD>, 256, 0)
-                         : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row<LOAD, FMT, RND, HAD>, 256, 0);
+    cudaError_t e;
+    if constexpr (WIDE) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row32<LOAD, FMT, RND, HAD>, 256, 0);
+    else e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_row<LOAD, FMT, RND, HAD>, 256, 0);
     v = (e == cudaSuccess && n >= 1) ? n : 1;
     cached[dev].store(v, std::memory_order_relaxed);   // every thread computes the same value
   }
@@ -36,8 +37,16 @@ int resident_blocks() {
 template <int LOAD, int FMT, int RND, int HAD>
 cudaError_t launch_one(const QParams& p, cudaStream_t s) {
   constexpr bool TRANS = LOAD == LD_TRANS || LOAD == LD_TRANS_FP4;
-  if constexpr ((TRANS && HAD > 128) || (RND == R_SQ16 && (HAD != 0 || LOAD == LD_ROW_FP4 || LOAD == LD_TRANS_FP4))) {
-    // a rotation block longer than the transposed kernel's 128-row tile;
+  if constexpr (LOAD == LD_ROW_F32) {
+    // an already transformed fp32 matrix: row-wise, 32-element tasks only
+    if (HAD != 0 || (p.cols % 32) != 0) return cudaErrorInvalidValue;
+    int64_t blocks = (p.rows * (p.cols >> 5) + 255) / 256;
+    const int64_t cap = int64_t(num_sms()) * resident_blocks<true, LOAD, FMT, RND, HAD>();
+    blocks = blocks > cap ? cap : (blocks < 1 ? 1 : blocks);
+    k_quant_row32<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
+    count_launch();
+    return cudaGetLastError();
+  } else if constexpr (RND == R_SQ16 && (HAD != 0 || LOAD == LD_ROW_FP4 || LOAD == LD_TRANS_FP4)) {
     // square blocks: bf16 input, no rotation
     return cudaErrorInvalidValue;
   } else {
@@ -51,8 +60,8 @@ cudaError_t launch_one(const QParams& p, cudaStream_t s) {
       k_quant_row32<LOAD, FMT, RND, HAD><<<dim3(unsigned(blocks)), 256, 0, s>>>(p);
       count_launch();
     } else if (wide) {
-      dim3 grid(unsigned((p.in_rows + TR_IN_ROWS - 1) / TR_IN_ROWS),
-                unsigned((p.in_cols + TR_IN_COLS - 1) / TR_IN_COLS));
+      using TT = T32Tile<HAD>;
+      dim3 grid(unsigned((p.in_rows + TT::ROWS - 1) / TT::ROWS), unsigned((p.in_cols + TT::COLS - 1) / TT::COLS));
       k_quant_trans32<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
       count_launch();
     } else if constexpr (HAD <= 16 && RND != R_SQ16) {

@@ -173,6 +173,78 @@ int fp4_quantize_mse(const void *x_dev, int64_t rows, int64_t cols, int32_t iter
 /* Bytes of the swizzled scale buffer for rows x n_groups scales. */
 size_t fp4_swizzled_scale_bytes(int64_t rows, int64_t n_groups);
 
+/* Dense orthonormal block transforms of the forward pass, [BG] appendix on
+ * linear transforms (Tables 13-14: Hadamard, DCT, DST and GSR at block sizes
+ * 16 to 256).  GSR is named but not defined by the pages and has no value
+ * here.
+ *   FP4_XFORM_DCT2: C[i][j] = f_i cos(pi (2j+1) i / (2k)), f_0 = sqrt(1/k),
+ *                   f_i = sqrt(2/k) (orthonormal DCT-II);
+ *   FP4_XFORM_DST2: S[i][j] = g_i sin(pi (2j+1)(i+1) / (2k)),
+ *                   g_{k-1} = sqrt(1/k), g_i = sqrt(2/k) (orthonormal DST-II).
+ * fp4_block_transform: y = M x for every k-block of every row of x, k =
+ * `block` in {16, 32, 64, 128, 256}.  x_dev: rows x cols bf16 row-major,
+ * y_dev: rows x cols fp32, both 16-byte aligned, caller-owned; cols a
+ * multiple of block, cols / block <= 65535.  y_i is the pairwise tree (level
+ * 0 adds j = 2m and 2m + 1) of the fp32 products fp32(M[i][j] x_j), every
+ * product and sum rounded to fp32; M's entries are fp64 values rounded once
+ * to fp32 (the cosine of the reduced angle pi m / (2k), m in [0, k], times
+ * the normalisation).  ws_dev: fp4_block_transform_workspace_size(block)
+ * bytes (the k x k fp32 matrix, rebuilt by each call), 16-byte aligned.
+ * Asynchronous on `stream`; 2 launches; an empty tensor launches nothing.
+ * Errors: FP4_ERR_UNSUPPORTED (kind, block), FP4_ERR_INVALID_ARG (shape,
+ * null pointers), FP4_ERR_ALIGNMENT, FP4_ERR_WORKSPACE, FP4_ERR_CUDA.  The
+ * workspace query returns 0 for an unsupported block. */
+enum fp4_transform_kind { FP4_XFORM_DCT2 = 1, FP4_XFORM_DST2 = 2 };
+size_t fp4_block_transform_workspace_size(int32_t block);
+int fp4_block_transform(const void *x_dev, float *y_dev, int64_t rows, int64_t cols, int32_t kind,
+                        int32_t block, void *ws_dev, size_t ws_bytes, fp4_stream_t stream);
+
+/* Quantise an fp32 matrix that is already transformed (e.g. the output of
+ * fp4_block_transform): fp4_quantize's rules with no rotation and no
+ * transpose.  y_dev: rows x cols fp32 row-major, 16-byte aligned, cols a
+ * multiple of 32.  rounding: RTN, QuEST, Four-Over-Six (NVFP4) or SR;
+ * MS-EDEN (its S lives on its own rotation blocks) and square blocks (bf16
+ * block maxima) return FP4_ERR_UNSUPPORTED.  out, seed, tensor_tag and the
+ * workspace (fp4_quantize_workspace_size(rows, cols, fmt, rounding, 0)) as
+ * for fp4_quantize. */
+int fp4_quantize_f32(const float *y_dev, int64_t rows, int64_t cols, int32_t fmt, int32_t rounding,
+                     int32_t group, uint64_t seed, uint32_t tensor_tag, fp4_qtensor *out,
+                     void *ws_dev, size_t ws_bytes, fp4_stream_t stream);
+
+/* MXFP4 with fitted scales (MXFP4-dagger), [BG] "MXFP Scale Fitting"
+ * (Appendix H, Table 11): the 8-bit scale of a 32-element group is a level q
+ * in [0, 255] standing for 2^(alpha q + L_min), L_min / L_max = log2 of the
+ * smallest / largest AbsMax group scale s = fp32(gmax / 6) of the tensor (over
+ * groups with s > 0), alpha = (L_max - L_min) / 255 (the page's fractional
+ * exponent step).  A group's level is the number of boundaries
+ * fp32(2^(L_min + alpha (k + 0.5))), k = 0..254, not above s; its elements
+ * are RTN_E2M1(x * fp32(1/d)), d = table[q] = fp32(2^(L_min + alpha q)),
+ * saturating at 6.  Exponents are fp64 (log2 / exp2 of CUDA's math library,
+ * each add and multiply rounded on its own), rounded once to fp32.  A group
+ * with s = 0 (or a non-finite reciprocal scale) gets level 0 and zero codes;
+ * with no s > 0 the table is all 1.  The scales are not powers of two, so the
+ * tensor cores' E8M0 block scaling cannot apply them: there is no GEMM for
+ * this format, only quantisation and de-quantisation (the page's accuracy
+ * use).
+ * fp4_quantize_mx_fit: x_dev bf16 rows x cols row-major (16-byte aligned),
+ * cols a multiple of 32 and of had_block; had_block in {0, 16, ..., 256}: the
+ * deterministic block Hadamard applied first (fp4_hadamard's transform).
+ * codes_dev rows x cols/2 (16-byte aligned), levels_dev rows x cols/32,
+ * table_dev 256 fp32: caller-owned outputs.  ws_dev:
+ * fp4_quantize_mx_fit_workspace_size() bytes, 16-byte aligned.  3 launches
+ * (+2 memsets); an empty tensor writes the all-1 table only.  A non-finite
+ * input sets FP4_ERR_NONFINITE_INPUT on the device.
+ * fp4_dequantize_mx_fit: out_dev[r][c] = fp32(E2M1(code) * table[level]),
+ * rows x cols fp32, 16-byte aligned.
+ * Errors: FP4_ERR_UNSUPPORTED (had_block), FP4_ERR_INVALID_ARG (shape, null
+ * pointers), FP4_ERR_ALIGNMENT, FP4_ERR_WORKSPACE, FP4_ERR_CUDA. */
+size_t fp4_quantize_mx_fit_workspace_size(void);
+int fp4_quantize_mx_fit(const void *x_dev, int64_t rows, int64_t cols, int32_t had_block,
+                        uint8_t *codes_dev, uint8_t *levels_dev, float *table_dev,
+                        void *ws_dev, size_t ws_bytes, fp4_stream_t stream);
+int fp4_dequantize_mx_fit(const uint8_t *codes_dev, const uint8_t *levels_dev, const float *table_dev,
+                          int64_t rows, int64_t cols, float *out_dev, fp4_stream_t stream);
+
 /* y = block (randomized) Hadamard of x along cols, fp32 out.
  * x_dev: rows x cols bf16; y_dev: rows x cols fp32; cols % block == 0.
  * [Q] "The Hadamard Transform": Sylvester order, 1/sqrt(g) normalisation. */
@@ -186,7 +258,7 @@ int fp4_hadamard(const void *x_dev, float *y_dev, int64_t rows, int64_t cols,
  * Complete Quartet II Computation Graph".  group must equal the format's
  * group size (16 NVFP4, 32 MXFP4).  cols must be a multiple of
  * max(group, had.block); with transpose = 1, in_cols must be a multiple of 8
- * and had.block at most 128 (FP4_ERR_UNSUPPORTED otherwise).
+ * (FP4_ERR_ALIGNMENT otherwise).
  * seed/tensor_tag key the Philox streams of SR (element index in the output
  * layout) and MS-EDEN (group index).  out: caller fills the pointers; the
  * call writes rows, cols and fmt.  ws_dev: fp4_quantize_workspace_size bytes,

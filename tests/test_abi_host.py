@@ -62,7 +62,7 @@ def quantize(lib, x, in_rows, in_cols, fmt, rnd, group, had=0, transpose=0, out=
     (1, 0, 16, 64, (64, 96), 0, INVALID),                    # ... nor of the rotation block
     (1, 0, 16, 0, (64, 36), 1, ALIGNMENT),                   # transposed: input rows of 36 (not 8k) elements
     (1, 0, 16, 0, (40, 64), 1, INVALID),                     # transposed inner dim 40 not a multiple of 16
-    (1, 0, 16, 256, (256, 64), 1, UNSUPPORTED),              # transposed: blocks up to 128
+    (1, 0, 16, 256, (256, 64), 1, WORKSPACE),                # transposed 256-blocks: valid, no workspace given
 ])
 def test_quantize_argument_checks(lib, fmt, rnd, group, had, shape, transpose, want):
     assert quantize(lib, FAKE, shape[0], shape[1], fmt, rnd, group, had, transpose) == want
@@ -204,3 +204,42 @@ def test_quantize_noalloc_square_block_limit(lib):
     assert lib.fp4_quantize_workspace_size(16384, 16384, 1, 5, 0) > 4 << 20
     empty = api.fp4_qtensor()
     assert _noalloc(lib, None, 0, 64, 1, 5, 16, out=empty) == OK
+
+
+def test_transform_and_fit_argument_checks(lib):
+    """fp4_block_transform, fp4_quantize_f32 and fp4_quantize_mx_fit return
+    their argument errors before any CUDA call."""
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    bt = lib.fp4_block_transform
+    bt.restype, bt.argtypes = ctypes.c_int, [P, P, I64, I64, I32, I32, P, SZ, P]
+    lib.fp4_block_transform_workspace_size.restype = SZ
+    lib.fp4_block_transform_workspace_size.argtypes = [I32]
+    assert lib.fp4_block_transform_workspace_size(256) == 256 * 256 * 4
+    assert lib.fp4_block_transform_workspace_size(48) == 0
+    assert bt(FAKE, FAKE, 8, 64, 3, 16, FAKE, 1 << 20, None) == UNSUPPORTED      # kind (GSR has no value)
+    assert bt(FAKE, FAKE, 8, 64, 1, 48, FAKE, 1 << 20, None) == UNSUPPORTED      # block
+    assert bt(FAKE, FAKE, 8, 80, 1, 32, FAKE, 1 << 20, None) == INVALID          # cols % block
+    assert bt(FAKE + 4, FAKE, 8, 64, 1, 16, FAKE, 1 << 20, None) == ALIGNMENT
+    assert bt(FAKE, FAKE, 8, 64, 2, 16, FAKE, 1023, None) == WORKSPACE           # needs 1024
+    assert bt(None, None, 0, 64, 1, 16, None, 0, None) == OK                      # empty
+    qf = lib.fp4_quantize_f32
+    qf.restype = ctypes.c_int
+    qf.argtypes = [P, I64, I64, I32, I32, I32, ctypes.c_uint64, ctypes.c_uint32,
+                   ctypes.POINTER(api.fp4_qtensor), P, SZ, P]
+    out = fake_out()
+    assert qf(FAKE, 8, 64, 1, 4, 16, 0, 0, ctypes.byref(out), FAKE, 1 << 20, None) == UNSUPPORTED   # MS-EDEN
+    assert qf(FAKE, 8, 64, 1, 5, 16, 0, 0, ctypes.byref(out), FAKE, 1 << 20, None) == UNSUPPORTED   # square
+    assert qf(FAKE, 8, 64, 0, 2, 32, 0, 0, ctypes.byref(out), FAKE, 1 << 20, None) == UNSUPPORTED   # MX 4/6
+    assert qf(FAKE, 8, 48, 1, 0, 16, 0, 0, ctypes.byref(out), FAKE, 1 << 20, None) == INVALID       # cols % 32
+    assert qf(FAKE + 8, 8, 64, 1, 0, 16, 0, 0, ctypes.byref(out), FAKE, 1 << 20, None) == ALIGNMENT
+    assert qf(FAKE, 8, 64, 1, 0, 16, 0, 0, ctypes.byref(out), None, 0, None) == WORKSPACE
+    mf = lib.fp4_quantize_mx_fit
+    mf.restype, mf.argtypes = ctypes.c_int, [P, I64, I64, I32, P, P, P, P, SZ, P]
+    lib.fp4_quantize_mx_fit_workspace_size.restype = SZ
+    assert lib.fp4_quantize_mx_fit_workspace_size() >= 256 + 255 * 4
+    assert mf(FAKE, 8, 64, 48, FAKE, FAKE, FAKE, FAKE, 4096, None) == UNSUPPORTED      # had block
+    assert mf(FAKE, 8, 48, 0, FAKE, FAKE, FAKE, FAKE, 4096, None) == INVALID            # cols % 32
+    assert mf(FAKE, 8, 64, 128, FAKE, FAKE, FAKE, FAKE, 4096, None) == INVALID          # cols % had
+    assert mf(FAKE, 8, 64, 0, FAKE, FAKE, FAKE, FAKE, 100, None) == WORKSPACE
+    assert mf(FAKE, 8, 64, 0, None, FAKE, FAKE, FAKE, 4096, None) == INVALID
+    assert mf(FAKE + 2, 8, 64, 0, FAKE, FAKE, FAKE, FAKE, 4096, None) == ALIGNMENT

@@ -34,8 +34,6 @@ def assert_qt_equal(g, o, check_mask=True):
 @pytest.mark.parametrize("fmt,rnd,had", COMBOS)
 @pytest.mark.parametrize("transpose", [False, True])
 def test_quantize_parity(cuda_lib, fmt, rnd, had, transpose):
-    if transpose and had > 128:
-        pytest.skip("rotation blocks above 128 are row-wise only")
     shape = (512, 200) if transpose else (200, 512)
     bits = syn.outlier_elements(shape, seed=7, stream=fmt * 10 + rnd)
     x = syn.bf16_bits_to_f32(bits)
@@ -67,6 +65,26 @@ def test_requantize_parity(cuda_lib, fmt, fwd_rnd, rnd, had, transpose):
                             transpose=transpose)
     o = qn.requantize(saved, rnd, had, had > 0, seed, 2, 4, transpose=transpose)
     assert_qt_equal(g, o)
+
+
+@pytest.mark.parametrize("fmt,fwd_rnd,rnd", [(qn.NVFP4, qn.FOUR_OVER_SIX, qn.MS_EDEN), (qn.NVFP4, qn.RTN, qn.SR),
+                                          (qn.MXFP4, qn.QUEST, qn.SR)])
+def test_requantize_transposed_256_blocks(cuda_lib, fmt, fwd_rnd, rnd):
+    """Re-quantisation of a saved tensor, transposed, with 256-element
+    rotation blocks (the transposed kernel's 256-row tile); 176 input
+    columns (NVFP4) leave a ragged last 32-column tile, MXFP4 groups need
+    224."""
+    cols = 176 if fmt == qn.NVFP4 else 224
+    bits = syn.student_t((512, cols), seed=4, unit_rms=True)
+    saved = qn.quantize(syn.bf16_bits_to_f32(bits), fmt, fwd_rnd, 0)
+    dev = cuda_lib.alloc_qtensor(512, cols, fmt, mask=False)
+    dev.codes.copy_(torch.from_numpy(fm.pack_codes(saved.codes)))
+    dev.scales.copy_(torch.from_numpy(saved.scales))
+    dev.tensor_scale.copy_(torch.tensor([float(saved.tensor_scale)], dtype=torch.float32))
+    g = cuda_lib.requantize(dev, rnd, 256, randomized=True, seed=91, sign_tag=1, tensor_tag=2, transpose=True)
+    o = qn.requantize(saved, rnd, 256, True, 91, 1, 2, transpose=True)
+    assert_qt_equal(g, o)
+    assert cuda_lib.get_last_error() == 0
 
 
 @pytest.mark.parametrize("block", [16, 32, 64, 128, 256])
@@ -204,11 +222,14 @@ def test_ms_eden_first_pass_bit_exact(cuda_lib, had, transpose):
     assert_qt_equal(g, o)
 
 
-def test_transposed_block_256_is_unsupported(cuda_lib):
-    x = to_dev(syn.gaussian((512, 256), 1.0, seed=1))
+def test_transposed_block_256_needs_whole_blocks(cuda_lib):
+    """Transposed 256-element rotation blocks run on the 256-row tile; the
+    quantised tensor's rows (the input's columns) run along the input's 384
+    rows, which do not hold whole 256-blocks."""
+    x = to_dev(syn.gaussian((384, 256), 1.0, seed=1))      # 384 input rows: not a multiple of 256
     with pytest.raises(cuda_lib.Fp4Error) as e:
         cuda_lib.quantize(x, qn.NVFP4, qn.RTN, 256, transpose=True)
-    assert e.value.status == 2                      # FP4_ERR_UNSUPPORTED
+    assert e.value.status == 1                      # FP4_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("transpose", [False, True])
