@@ -272,6 +272,94 @@ def transpose_square16(qt, linear=True, swizzled=True, out=None):
     return out
 
 
+XFORM_DCT2, XFORM_DST2 = 1, 2
+
+
+def block_transform(x, kind, block, out=None, ws=None):
+    """fp4_block_transform: the orthonormal DCT-II / DST-II of every
+    `block`-element block of x's rows (bf16 in, fp32 out)."""
+    lib = load()
+    lib.fp4_block_transform_workspace_size.restype = ctypes.c_size_t
+    lib.fp4_block_transform_workspace_size.argtypes = [ctypes.c_int32]
+    f = lib.fp4_block_transform
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                  ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = alloc_workspace(lib.fp4_block_transform_workspace_size(block), x.device)
+    _check(f(_ptr(x), _ptr(out), x.shape[0], x.shape[1], kind, block, _ptr(ws), ws.numel(), _stream()),
+           "fp4_block_transform")
+    return out
+
+
+def quantize_f32(y, fmt, rnd, seed=0, tensor_tag=0, linear=True, swizzled=True, out=None, ws=None):
+    """fp4_quantize_f32: quantise an already transformed fp32 CUDA tensor."""
+    lib = load()
+    f = lib.fp4_quantize_f32
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_uint64, ctypes.c_uint32, ctypes.POINTER(fp4_qtensor), ctypes.c_void_p, ctypes.c_size_t,
+                  ctypes.c_void_p]
+    assert y.dtype == torch.float32 and y.is_cuda and y.dim() == 2 and y.is_contiguous()
+    rows, cols = y.shape
+    if out is None:
+        out = alloc_qtensor(rows, cols, fmt, linear, swizzled, mask=(rnd == QUEST), device=y.device)
+    if ws is None:
+        ws = alloc_workspace(workspace_size(rows, cols, fmt, rnd, 0), y.device)
+    cs = out.c_struct()
+    _check(f(_ptr(y), rows, cols, fmt, rnd, GROUP[fmt], seed, tensor_tag, ctypes.byref(cs), _ptr(ws), ws.numel(),
+             _stream()), "fp4_quantize_f32")
+    return out
+
+
+@dataclass
+class FitTensor:
+    """MXFP4 with fitted scales: codes, one level per 32 elements, the
+    tensor's 256-entry scale table."""
+    codes: torch.Tensor
+    levels: torch.Tensor
+    table: torch.Tensor
+
+
+def quantize_mx_fit(x, had_block=0, ws=None):
+    """fp4_quantize_mx_fit (MXFP4-dagger) of a bf16 CUDA tensor."""
+    lib = load()
+    lib.fp4_quantize_mx_fit_workspace_size.restype = ctypes.c_size_t
+    lib.fp4_quantize_mx_fit_workspace_size.argtypes = []
+    f = lib.fp4_quantize_mx_fit
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
+    rows, cols = x.shape
+    ft = FitTensor(torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device),
+                   torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device),
+                   torch.empty((256,), dtype=torch.float32, device=x.device))
+    if ws is None:
+        ws = alloc_workspace(lib.fp4_quantize_mx_fit_workspace_size(), x.device)
+    _check(f(_ptr(x), rows, cols, had_block, _ptr(ft.codes), _ptr(ft.levels), _ptr(ft.table), _ptr(ws), ws.numel(),
+             _stream()), "fp4_quantize_mx_fit")
+    return ft
+
+
+def dequantize_mx_fit(ft, out=None):
+    """fp4_dequantize_mx_fit: fp32(E2M1(code) * table[level])."""
+    lib = load()
+    f = lib.fp4_dequantize_mx_fit
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    rows, cols = ft.codes.shape[0], ft.codes.shape[1] * 2
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float32, device=ft.codes.device)
+    _check(f(_ptr(ft.codes), _ptr(ft.levels), _ptr(ft.table), rows, cols, _ptr(out), _stream()),
+           "fp4_dequantize_mx_fit")
+    return out
+
+
 def hadamard(x, block, randomized=False, seed=0, sign_tag=0):
     lib = load()
     y = torch.empty(x.shape, dtype=torch.float32, device=x.device)

@@ -17,7 +17,9 @@ namespace fp4 {
 enum : int { FMT_MX = 0, FMT_NV = 1 };
 // R_AMAX: the global amax pass; R_SQ16: RTN against 16 x 16 block maxima.
 enum : int { R_RTN = 0, R_QUEST = 1, R_FOS = 2, R_SR = 3, R_EDEN = 4, R_AMAX = 5, R_SQ16 = 6 };
-enum : int { LD_ROW = 0, LD_TRANS = 1, LD_ROW_FP4 = 2, LD_TRANS_FP4 = 3 };
+// LD_ROW_F32: an fp32 matrix that is already transformed (row-wise, 32-element
+// tasks only; fp4_quantize_f32).
+enum : int { LD_ROW = 0, LD_TRANS = 1, LD_ROW_FP4 = 2, LD_TRANS_FP4 = 3, LD_ROW_F32 = 4 };
 
 struct QParams {
   // input: bf16 matrix, or a saved FP4 tensor (codes + linear scales + scale)
