@@ -497,14 +497,18 @@ __global__ void __launch_bounds__(THREADS, 1)
 // read both CTAs' shared memory, and each CTA keeps its 128 x 256 half of the
 // accumulator in its own tensor memory.  Each CTA thus moves half the B
 // bytes per MMA of the one-CTA kernel, which buys two more pipeline stages.
-//   operands: both CTAs' TMA loads complete on the leader's full[s]
-//             (expected bytes set by the leader's producer);
-//   scales:   each CTA loads its own scale atoms (its 128 A rows, all 256 B
-//             rows) and its stagers write its own TMEM, then arrive on the
-//             leader's sf_full[b];
-//   releases: the leader's commits arrive on empty[s], sf_empty[b] and
-//             acc_full in both CTAs (tcgen05.commit multicast);
+//   operands: both CTAs' TMA loads (warp 0) complete on the leader's
+//             full[s] (expected bytes set by the leader's producer);
+//   scales:   each CTA copies its own scale atoms (its 128 A rows, all 256 B
+//             rows; warp 3) into its sf_ld[s], and its stagers write them
+//             into TMEM scale buffer s, then arrive on the leader's full[s]
+//             (one producer arrival + 8 stager-warp arrivals + the bytes);
+//   releases: the leader's commits arrive on empty[s] and acc_full in both
+//             CTAs (tcgen05.commit multicast);
 //   epilogue: each CTA drains its half and arrives on the leader's acc_empty.
+// The leader's MMA thread thus waits on one barrier and commits one release
+// per k-tile: its own instruction stream, not the tensor pipe, sets the pace
+// when it has more to do per k-tile.
 namespace pair {
 
 constexpr int STAGES = 5;
@@ -523,6 +527,7 @@ constexpr int PTHREADS = 512;
 constexpr int REG_CTRL = 56, REG_STAGE = 80, REG_EPI = 184;
 static_assert(128 * (REG_CTRL + REG_STAGE + 2 * REG_EPI) <= 65536, "register split of the CTA-pair kernel");
 static_assert(SMEM_BYTES <= 232448, "shared memory of the CTA-pair kernel");
+static_assert(SF_COL + STAGES * SF_BUF_COLS <= TMEM_COLS, "one scale TMEM buffer per stage");
 
 __device__ __forceinline__ uint32_t cta_rank() {
   uint32_t r;
@@ -675,14 +680,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
   uint8_t* sSFA = sB + STAGES * B_BYTES;
   uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
   uint8_t* sStage = sSFB + STAGES * SFB_BYTES;
+  // Stage s owns an operand slot, a scale slot and scale TMEM buffer s.
   uint64_t* full = reinterpret_cast<uint64_t*>(sStage + 2 * STG_BYTES);   // leader: operand bytes of both CTAs
-  uint64_t* empty = full + STAGES;                                          // both: slot consumed by the MMAs
+                                                                            // + 4 stager warps x 2 CTAs
+  uint64_t* empty = full + STAGES;                                          // both: stage consumed by the MMAs
   uint64_t* sf_ld = empty + STAGES;                                         // both: this CTA's scale atoms landed
   uint64_t* acc_full = sf_ld + STAGES;                                      // both
   uint64_t* acc_empty = acc_full + 1;                                       // leader: 4 warps x 2 CTAs
-  uint64_t* sf_full = acc_empty + 1;                                        // leader: 4 warps x 2 CTAs (x NSF)
-  uint64_t* sf_empty = sf_full + NSF;                                       // both
-  uint64_t* drain = sf_empty + NSF;                                         // leader: MMAs retired
+  uint64_t* drain = acc_empty + 1;                                          // leader: MMAs retired
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -696,13 +701,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 8);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_ld[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 16);
-    for (int b = 0; b < NSF; ++b) { mbar_init(&sf_full[b], 8); mbar_init(&sf_empty[b], 1); }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -724,11 +728,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
 
   if (wg == 0) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CTRL));
-  if (warp == 0 && lane == 0) {
-    // ------------------------------------------------------ TMA producer --
+  if ((warp == 0 || warp == 3) && lane == 0) {
+    // --------------------------------------------- producers (2 threads) --
+    // Warp 0 loads the operand tiles (TMA, completing on the leader's
+    // full[s]), warp 3 this CTA's scale atoms (bulk copies, on its own
+    // sf_ld[s]): one thread issuing every copy of a k-tile is itself the
+    // bottleneck at this rate.  Both walk the same stages and wait for the
+    // same releases.
+    const bool operands = warp == 0;
     int s = 0;
     uint32_t ph = 0;
     const int64_t nrb_a = (p.M + 127) / 128, nrb_b = (p.N + 127) / 128;
+    const int nk = int(nkt);
+    const int last_mma = int((p.K - int64_t(nk - 1) * BK) / 64);
+    int* const st = p.status;
+    const int64_t nkb = p.nkb;
+    const uint8_t* const sfa_g = p.sfa;
+    const uint8_t* const sfb_g = p.sfb;
     for (int64_t t = pair_id; t < ntiles && !*abort_flag; t += npairs) {
       int64_t mb, nb;
       tile_coords2(t, nm, nn, p.raster, mb, nb);
@@ -736,21 +752,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
       // 128-row halves that exist (a half entirely past M or N is not loaded)
       const int a_halves = (mb * 2 + 1 < nrb_a) ? 2 : 1, b_halves = (nb * 2 + 1 < nrb_b) ? 2 : 1;
       const bool load_a = ra < nrb_a, load_b = rb < nrb_b;
-      for (int64_t kt = 0; kt < nkt; ++kt) {
-        if (!wait_c(&empty[s], ph ^ 1, abort_flag, p.status)) break;
-        const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
-        const int n_mma = kel / 64;
-        const int atoms = FMT == 1 ? n_mma : (n_mma + 1) / 2;
-        const int64_t atom0 = kt * (BK / G / 4);
-        if (leader) mbar_expect_tx(&full[s], uint32_t((a_halves + b_halves) * A_BYTES));
-        if (load_a) tma_load_pair(sA + s * A_BYTES, &map_a, int(kt * (BK / 2)), int(ra * 128), &full[s]);
-        if (load_b) tma_load_pair(sB + s * B_BYTES, &map_b, int(kt * (BK / 2)), int(rb * 128), &full[s]);
-        const uint32_t sf_bytes = uint32_t(atoms) * 512u * uint32_t((load_a ? 1 : 0) + b_halves);
-        mbar_expect_tx(&sf_ld[s], sf_bytes);
-        if (load_a) bulk_load(sSFA + s * SFA_BYTES, p.sfa + (ra * p.nkb + atom0) * 512, atoms * 512u, &sf_ld[s]);
-        for (int r = 0; r < b_halves; ++r)
-          bulk_load(sSFB + s * SFB_BYTES + r * 4 * 512, p.sfb + ((nb * 2 + r) * p.nkb + atom0) * 512,
-                    atoms * 512u, &sf_ld[s]);
+      const uint32_t op_bytes = uint32_t((a_halves + b_halves) * A_BYTES);
+      const uint8_t* const sfa_row = sfa_g + ra * nkb * 512;
+      const uint8_t* const sfb_row0 = sfb_g + (nb * 2) * nkb * 512;
+      for (int kt = 0; kt < nk; ++kt) {
+        if (!wait_c(&empty[s], ph ^ 1, abort_flag, st)) break;
+        if (operands) {
+          if (leader) mbar_expect_tx(&full[s], op_bytes);
+          if (load_a) tma_load_pair(sA + s * A_BYTES, &map_a, kt * (BK / 2), int(ra * 128), &full[s]);
+          if (load_b) tma_load_pair(sB + s * B_BYTES, &map_b, kt * (BK / 2), int(rb * 128), &full[s]);
+        } else {
+          const int n_mma = kt + 1 < nk ? BK / 64 : last_mma;
+          const uint32_t abytes = uint32_t(FMT == 1 ? n_mma : (n_mma + 1) / 2) * 512u;
+          const int64_t off = int64_t(kt) * (BK / G / 4) * 512;
+          mbar_expect_tx(&sf_ld[s], abytes * uint32_t((load_a ? 1 : 0) + b_halves));
+          if (load_a) bulk_load(sSFA + s * SFA_BYTES, sfa_row + off, abytes, &sf_ld[s]);
+          for (int r = 0; r < b_halves; ++r)
+            bulk_load(sSFB + s * SFB_BYTES + r * 4 * 512, sfb_row0 + r * nkb * 512 + off, abytes, &sf_ld[s]);
+        }
         if (++s == STAGES) { s = 0; ph ^= 1; }
       }
     }
@@ -760,38 +779,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // --------------------------------------------------------- MMA issue --
-    int s = 0, buf = 0;
+    // One thread issues every MMA, and its own scalar work per loop trip
+    // (counters, descriptors, parameter loads) costs about as much as the
+    // four MMAs of a k-tile take on the tensor pipe.  So the loop is lean: all
+    // bases are in registers, counters are 32-bit, and each trip takes two
+    // k-tiles (each waited for, issued and released on its own).
+    int s = 0;
     uint32_t ph = 0, acc_ph = 0;
-    uint32_t sph = 0;
     bool ok = true, issued = false;
-    for (int64_t t = pair_id; ok && t < ntiles && !*abort_flag; t += npairs) {
-      if (!wait_c(acc_empty, acc_ph ^ 1, abort_flag, p.status)) break;
+    const int nk = int(nkt);
+    const int last_mma = int((p.K - int64_t(nk - 1) * BK) / 64);   // MMAs of the last k-tile
+    int* const st = p.status;
+    const uint64_t ad0 = desc_sw128(smem_u32(sA)), bd0 = desc_sw128(smem_u32(sB));
+    const uint32_t id0 = idesc(FMT, BN, 256, 0, 0), acc_t = tmem + ACC_COL, sf0 = tmem + SF_COL;
+    // Waits for stage s (operands of both CTAs and the scales in TMEM),
+    // issues k-tile kt from it and releases it; false when the wait gave up.
+    auto ktile = [&](int kt) -> bool {
+      if (!wait_c(&full[s], ph, abort_flag, st)) return false;
       tc_fence_after();
-      for (int64_t kt = 0; kt < nkt; ++kt) {
-        if (!wait_c(&full[s], ph, abort_flag, p.status)) { ok = false; break; }
-        if (!wait_c(&sf_full[buf], sph, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const int kel = int(p.K - kt * BK < BK ? p.K - kt * BK : BK);
-        const int n_mma = kel / 64;
-        const uint64_t ad = desc_sw128(smem_u32(sA + s * A_BYTES)), bd = desc_sw128(smem_u32(sB + s * B_BYTES));
-        const uint32_t sfbase = tmem + SF_COL + SF_BUF_COLS * uint32_t(buf);
-        if (n_mma == BK / 64) {
-          mma_ktile<FMT, BK / 64, true>(tmem + ACC_COL, ad, bd, sfbase, idesc(FMT, BN, 256, 0, 0), kt > 0);
-        } else {                                          // the last, partial k-tile
-          for (int kk = 0; kk < n_mma; ++kk) {
-            const int atom = FMT == 1 ? kk : kk / 2;
-            const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
-            mma_pair<FMT>(tmem + ACC_COL, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc(FMT, BN, 256, sf_id, sf_id),
-                          (sfbase + 4 * atom) | (sf_id << 30), (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30),
-                          (kt > 0 || kk > 0) ? 1u : 0u);
-          }
+      const uint64_t ad = ad0 + uint64_t(s * (A_BYTES >> 4)), bd = bd0 + uint64_t(s * (B_BYTES >> 4));
+      const uint32_t sfbase = sf0 + SF_BUF_COLS * uint32_t(s);
+      if (kt + 1 < nk || last_mma == BK / 64) {
+        mma_ktile<FMT, BK / 64, true>(acc_t, ad, bd, sfbase, id0, kt > 0);
+      } else {                                        // the last, partial k-tile
+        for (int kk = 0; kk < last_mma; ++kk) {
+          const int atom = FMT == 1 ? kk : kk / 2;
+          const uint32_t sf_id = FMT == 1 ? 0u : uint32_t(kk & 1) * 2u;
+          mma_pair<FMT>(acc_t, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc(FMT, BN, 256, sf_id, sf_id),
+                        (sfbase + 4 * atom) | (sf_id << 30), (sfbase + SFB_OFF + 8 * atom) | (sf_id << 30),
+                        (kt > 0 || kk > 0) ? 1u : 0u);
         }
-        issued = true;
-        commit_both(&empty[s]);
-        commit_both(&sf_empty[buf]);
-        if (kt == nkt - 1) commit_both(acc_full);
-        if (++buf == NSF) { buf = 0; sph ^= 1; }
-        if (++s == STAGES) { s = 0; ph ^= 1; }
+      }
+      commit_both(&empty[s]);
+      if (kt == nk - 1) commit_both(acc_full);
+      if (++s == STAGES) { s = 0; ph ^= 1; }
+      return true;
+    };
+    for (int64_t t = pair_id; ok && t < ntiles && !*abort_flag; t += npairs) {
+      if (!wait_c(acc_empty, acc_ph ^ 1, abort_flag, st)) break;
+      tc_fence_after();
+      issued = true;
+      for (int kt = 0; kt < nk; kt += 2) {
+        if (!ktile(kt)) { ok = false; break; }
+        if (kt + 1 < nk && !ktile(kt + 1)) { ok = false; break; }
       }
       acc_ph ^= 1;
     }
@@ -804,15 +834,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
   } else if (wg == 1) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_STAGE));
     // ------------------------------------------- scale factors -> TMEM --
+    // Scale buffer s is free once stage s's scale atoms have landed: the
+    // producer issued their copies after the MMAs that last read buffer s
+    // released the stage.  Each stager warp arrives on the leader's full[s].
     const int q = warp & 3;
-    int s = 0, buf = 0;
+    int s = 0;
     uint32_t ph = 0;
-    uint32_t sph = 0;
     bool ok = true;
+    const uint32_t full_l = mapa(full, 0);
     for (int64_t t = pair_id; ok && t < ntiles; t += npairs) {
       for (int64_t kt = 0; kt < nkt; ++kt) {
-        const bool a = wait_c(&sf_empty[buf], sph ^ 1u, abort_flag, p.status);
-        const bool b = a && wait_c(&sf_ld[s], ph, abort_flag, p.status);
+        const bool b = wait_c(&sf_ld[s], ph, abort_flag, p.status);
         if (__any_sync(0xFFFFFFFFu, !b)) { ok = false; break; }
         tc_fence_after();
         uint32_t va[16], vb[32];
@@ -829,7 +861,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
             vb[o] = y.x; vb[o + 1] = y.y; vb[o + 2] = y.z; vb[o + 3] = y.w;
           }
         }
-        const uint32_t base = tmem + (uint32_t(q * 32) << 16) + SF_COL + SF_BUF_COLS * uint32_t(buf);
+        const uint32_t base = tmem + (uint32_t(q * 32) << 16) + SF_COL + SF_BUF_COLS * uint32_t(s);
         asm volatile(
             "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(base),
             "r"(va[0]), "r"(va[1]), "r"(va[2]), "r"(va[3]), "r"(va[4]), "r"(va[5]), "r"(va[6]), "r"(va[7]), "r"(va[8]),
@@ -844,8 +876,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_cluster(mapa(&sf_full[buf], 0));
-        if (++buf == NSF) { buf = 0; sph ^= 1; }
+        if (lane == 0) arrive_cluster(full_l + uint32_t(s) * 8u);
         if (++s == STAGES) { s = 0; ph ^= 1; }
       }
     }
