@@ -120,6 +120,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -672,7 +680,8 @@ __device__ __forceinline__ void tile_coords2(int64_t t, int64_t nm, int64_t nn, 
 template <int FMT, int OUT, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                const __grid_constant__ CUtensorMap map_d, Params p) {
+                const __grid_constant__ CUtensorMap map_d, const __grid_constant__ CUtensorMap map_sfa,
+                const __grid_constant__ CUtensorMap map_sfb, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -740,11 +749,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
     uint32_t ph = 0;
     const int64_t nrb_a = (p.M + 127) / 128, nrb_b = (p.N + 127) / 128;
     const int nk = int(nkt);
-    const int last_mma = int((p.K - int64_t(nk - 1) * BK) / 64);
     int* const st = p.status;
-    const int64_t nkb = p.nkb;
-    const uint8_t* const sfa_g = p.sfa;
-    const uint8_t* const sfb_g = p.sfb;
     for (int64_t t = pair_id; t < ntiles && !*abort_flag; t += npairs) {
       int64_t mb, nb;
       tile_coords2(t, nm, nn, p.raster, mb, nb);
@@ -753,8 +758,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
       const int a_halves = (mb * 2 + 1 < nrb_a) ? 2 : 1, b_halves = (nb * 2 + 1 < nrb_b) ? 2 : 1;
       const bool load_a = ra < nrb_a, load_b = rb < nrb_b;
       const uint32_t op_bytes = uint32_t((a_halves + b_halves) * A_BYTES);
-      const uint8_t* const sfa_row = sfa_g + ra * nkb * 512;
-      const uint8_t* const sfb_row0 = sfb_g + (nb * 2) * nkb * 512;
       for (int kt = 0; kt < nk; ++kt) {
         if (!wait_c(&empty[s], ph ^ 1, abort_flag, st)) break;
         if (operands) {
@@ -762,13 +765,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
           if (load_a) tma_load_pair(sA + s * A_BYTES, &map_a, kt * (BK / 2), int(ra * 128), &full[s]);
           if (load_b) tma_load_pair(sB + s * B_BYTES, &map_b, kt * (BK / 2), int(rb * 128), &full[s]);
         } else {
-          const int n_mma = kt + 1 < nk ? BK / 64 : last_mma;
-          const uint32_t abytes = uint32_t(FMT == 1 ? n_mma : (n_mma + 1) / 2) * 512u;
-          const int64_t off = int64_t(kt) * (BK / G / 4) * 512;
-          mbar_expect_tx(&sf_ld[s], abytes * uint32_t((load_a ? 1 : 0) + b_halves));
-          if (load_a) bulk_load(sSFA + s * SFA_BYTES, sfa_row + off, abytes, &sf_ld[s]);
-          for (int r = 0; r < b_halves; ++r)
-            bulk_load(sSFB + s * SFB_BYTES + r * 4 * 512, sfb_row0 + r * nkb * 512 + off, abytes, &sf_ld[s]);
+          // Scale atoms through 3-D views {128 words, atom, 128-row block} of
+          // the tensor-core scale layout: 4 atoms of this CTA's A rows, and
+          // 4 atoms x both 128-row blocks of the tile's B rows, in one copy
+          // each (atoms past the last, or a B block past N, read as zeros).
+          const int atom0 = kt * (BK / G / 4);
+          mbar_expect_tx(&sf_ld[s], uint32_t(load_a ? SFA_BYTES : 0) + uint32_t(SFB_BYTES));
+          if (load_a) tma_load_3d(sSFA + s * SFA_BYTES, &map_sfa, 0, atom0, int(ra), &sf_ld[s]);
+          tma_load_3d(sSFB + s * SFB_BYTES, &map_sfb, 0, atom0, int(nb * 2), &sf_ld[s]);
         }
         if (++s == STAGES) { s = 0; ph ^= 1; }
       }
@@ -1034,6 +1038,22 @@ static bool make_map_d(CUtensorMap* m, void* D, int64_t M, int64_t N, int out_dt
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor-core scale layout of a rows x groups scale matrix as a 3-D tensor
+// of 32-bit words {128 words of an atom, nkb atoms of a 128-row block, row
+// blocks}; box {128, 4, box_blocks} (4 atoms: one k-tile of 256 elements for
+// NVFP4, two for MXFP4); reads past the end return zeros.
+static bool make_map_sf(CUtensorMap* m, const uint8_t* swz, int64_t rows, int64_t nkb, int box_blocks) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, cuuint64_t(nkb), cuuint64_t((rows + 127) / 128)};
+  cuuint64_t strides[2] = {512, cuuint64_t(nkb) * 512};
+  cuuint32_t box[3] = {128, 4, cuuint32_t(box_blocks)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(swz), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int FMT, int OUT, int EPI>
 static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
                           cudaStream_t s) {
@@ -1058,6 +1078,8 @@ static cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CU
 template <int FMT, int OUT, int EPI>
 static cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md,
                                const Params& p, cudaStream_t s) {
+  CUtensorMap msa, msb;
+  if (!make_map_sf(&msa, p.sfa, p.M, p.nkb, 1) || !make_map_sf(&msb, p.sfb, p.N, p.nkb, 2)) return cudaErrorInvalidValue;
   auto kern = pair::k_gemm_pair<FMT, OUT, EPI>;
   static std::atomic<int> max_clusters[64] = {};
   int dev = 0;
@@ -1081,7 +1103,7 @@ static cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, con
   }
   const int64_t tiles = ((p.M + 255) / 256) * ((p.N + BN - 1) / BN);
   const int64_t pairs = tiles < mc ? tiles : mc;
-  kern<<<unsigned(2 * pairs), pair::PTHREADS, pair::SMEM_BYTES, s>>>(ma, mb, md, p);
+  kern<<<unsigned(2 * pairs), pair::PTHREADS, pair::SMEM_BYTES, s>>>(ma, mb, md, msa, msb, p);
   count_launch();
   return cudaGetLastError();
 }
