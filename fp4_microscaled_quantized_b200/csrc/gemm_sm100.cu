@@ -222,6 +222,20 @@ template <int FMT, int NK, bool PAIR = false>
 __device__ __forceinline__ void mma_ktile(uint32_t acc, uint64_t ad, uint64_t bd, uint32_t sfbase, uint32_t idesc0,
                                           bool accumulate);
 
+// The same load without its wait (several loads, then one tcgen05.wait::ld).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
   asm volatile(
@@ -916,7 +930,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
       tc_fence_after();
       float v[128];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tmem_ld32(tmem + ACC_COL + (uint32_t(q * 32) << 16) + 128 * h + 32 * i, v + 32 * i);
+      for (int i = 0; i < 4; ++i) tmem_ld32_async(tmem + ACC_COL + (uint32_t(q * 32) << 16) + 128 * h + 32 * i, v + 32 * i);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       tc_fence_before();
       __syncwarp();
       if (lane == 0) arrive_cluster(acc_empty_l);
