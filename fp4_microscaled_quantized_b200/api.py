@@ -485,12 +485,12 @@ def selftest_e2m1():
 
 def selftest_arith():
     """Mismatch counts of the quantisers' exact division by 6, E8M3
-    reciprocal, per-tensor division, E4M3 decoder and E4M3 encoder against
-    CUDA's IEEE operations (all 0 expected)."""
+    reciprocal, per-tensor division, E4M3 decoder, E4M3 encoder and MS-EDEN
+    pseudo-scale rounding against CUDA's IEEE operations (all 0 expected)."""
     lib = load()
     lib.fp4_selftest_arith.restype = ctypes.c_int
     lib.fp4_selftest_arith.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
-    cnt = torch.zeros((5,), dtype=torch.int64, device="cuda")
+    cnt = torch.zeros((6,), dtype=torch.int64, device="cuda")
     _check(lib.fp4_selftest_arith(_ptr(cnt), _stream()), "fp4_selftest_arith")
     return [int(v) for v in cnt.cpu()]
 

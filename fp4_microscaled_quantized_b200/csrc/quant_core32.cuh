@@ -39,6 +39,19 @@ __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t b) {
   return h;
 }
 
+// E2M1 RTN of two values as in e2m1x2_rn, returning also their grid values
+// as f16x2 (exact), decoded from the same one-byte code inside the asm block.
+__device__ __forceinline__ uint32_t e2m1x2_rn_dec(float lo, float hi, uint32_t& h) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t.reg .b16 s;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %3, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, t;\n\t"
+      "mov.b16 s, {t, 0};\n\t"
+      "cvt.u32.u16 %0, s;\n\t}"
+      : "=r"(r), "=r"(h) : "f"(lo), "f"(hi));
+  return r;
+}
+
 // Clear negative-zero codes (a value rounding to 0 is stored as +0).
 __device__ __forceinline__ uint32_t clear_neg_zero(uint32_t w) {
   const uint32_t nz = ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;  // bit 3 set iff mag != 0
@@ -125,6 +138,49 @@ __device__ __forceinline__ void enc16(const float* x, float inv, bool ok, uint32
   enc16_raw(x, inv, ok, w);
   w[0] = clear_neg_zero(w[0]);
   w[1] = clear_neg_zero(w[1]);
+}
+
+// enc8_raw of v together with the signed grid values q of the 8 codes
+// (code 8 gives -0), without unpacking the word again.
+__device__ __forceinline__ uint32_t enc8_dec(const float* v, float* q) {
+  uint32_t b[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t h;
+    b[k] = e2m1x2_rn_dec(v[2 * k], v[2 * k + 1], h);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    q[2 * k] = f.x;
+    q[2 * k + 1] = f.y;
+  }
+  const uint32_t lo = __byte_perm(b[0], b[1], 0x0040u);
+  const uint32_t hi = __byte_perm(b[2], b[3], 0x0040u);
+  return __byte_perm(lo, hi, 0x5410u);
+}
+
+// enc16_raw with the grid values of the 16 codes (all zero when !ok).
+__device__ __forceinline__ void enc16_dec(const float* x, float inv, bool ok, uint32_t* w, float* q) {
+  float v[16];
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) st2(v, j, __fmul2_rn(ld2(x, j), splat2(inv)));
+  w[0] = enc8_dec(v, q);
+  w[1] = enc8_dec(v + 8, q + 8);
+  if (!ok) {
+    w[0] = w[1] = 0u;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) q[j] = 0.0f;
+  }
+}
+
+// sse16 from grid values already decoded.
+__device__ __forceinline__ float sse16q(const float* x, const float* q, float d) {
+  float s[16];
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    const float2 qd = __fmul2_rn(ld2(q, j), splat2(d));
+    const float2 e = make_float2(__fsub_rn(x[j], qd.x), __fsub_rn(x[j + 1], qd.y));
+    st2(s, j, __fmul2_rn(e, e));
+  }
+  return tree16p(s);
 }
 
 // Signed grid values of the 8 codes of a word (element j from bits 4j..4j+3):
@@ -223,6 +279,17 @@ __device__ __forceinline__ void fwht32_lanes(float* x, int lane) {
   for (int j = 0; j < 32; j += 2) st2(x, j, __fmul2_rn(ld2(x, j), splat2(c)));
 }
 
+// e8m3_round(fp32(g / 6)) for g >= 0 or NaN.  The product with fp32(1/6)
+// (relative error 2^-25) lies within 1.5 ulp of g / 6, so its bit pattern is
+// within one of the correctly rounded quotient's and the E8M3 rounding of
+// the two differs only when the product's low 20 bits lie within two of the
+// rounding midpoint 0x80000; only then is the quotient divided exactly.
+__device__ __forceinline__ float e8m3_div6(float g) {
+  const float q = __fmul_rn(g, 0.166666672f);
+  if (((fbits(q) + 2u - 0x80000u) & 0xFFFFFu) <= 4u) return e8m3_round(__fdiv_rn(g, 6.0f));
+  return e8m3_round(q);
+}
+
 // Per-tensor constants of the NVFP4 scale rules, computed once per thread:
 // the tensor scale and the divisions of the group maximum by the largest
 // normalised value times it.
@@ -296,9 +363,11 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
         const float d6 = __fmul_rn(v2.x, s32), i6 = __frcp_rn(d6);
         const float d4 = __fmul_rn(v2.y, s32), i4 = __frcp_rn(d4);
         uint32_t w6[2], w4[2];
-        enc16_raw(xg, i6, finite_pos(d6, i6), w6);
-        enc16_raw(xg, i4, finite_pos(d4, i4), w4);
-        const bool pick4 = sse16(xg, w4, d4) < sse16(xg, w6, d6);   // a tie keeps the 6-scale
+        float q[16];
+        enc16_dec(xg, i6, finite_pos(d6, i6), w6, q);
+        const float e6 = sse16q(xg, q, d6);
+        enc16_dec(xg, i4, finite_pos(d4, i4), w4, q);
+        const bool pick4 = sse16q(xg, q, d4) < e6;   // a tie keeps the 6-scale
         wg[0] = clear_neg_zero(pick4 ? w4[0] : w6[0]);
         wg[1] = clear_neg_zero(pick4 ? w4[1] : w6[1]);
         sb[g] = pick4 ? (c2 >> 8) : (c2 & 0xFFu);
@@ -364,12 +433,14 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
       const float* xg = x + 16 * g;
-      const float pq = e8m3_round(exact_div(bitsf(gmb[g]), qc.d6));
+      const float pq = e8m3_div6(bitsf(gmb[g]));
       const float inv = rcp_e8m3(pq);
-      enc16(xg, inv, finite_pos(pq, inv), w + 2 * g);
+      // grid values of the raw codes: a -0 instead of +0 changes only the
+      // sign of zero terms, hence of an all-zero sum, which gives S = 1 either way
       float q[16], yy[16], yq[16];
-      dec8(w[2 * g], q);
-      dec8(w[2 * g + 1], q + 8);
+      enc16_dec(xg, inv, finite_pos(pq, inv), w + 2 * g, q);
+      w[2 * g] = clear_neg_zero(w[2 * g]);
+      w[2 * g + 1] = clear_neg_zero(w[2 * g + 1]);
 #pragma unroll
       for (int j = 0; j < 16; j += 2) {
         const float2 y2 = ld2(xg, j);
@@ -489,20 +560,23 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
   return lmax;
 }
 
-// Resident 256-thread blocks per SM the register allocation is held to: the
-// kernels are issue bound, and one more resident block pays for a few spilled
-// registers in RTN / amax (4 blocks) and Four-Over-Six / MS-EDEN (3 blocks);
+// Resident 256-thread blocks per SM the register allocation is held to.  The
+// row kernels hold the next task's 64 input bytes in registers while they
+// process the current one: RTN / amax at 3 blocks (85 registers) and
+// Four-Over-Six / MS-EDEN at 2 (128) run faster that way than at 4 / 3
+// blocks, with or without the early load (which spills at those budgets);
 // SR and QuEST keep their registers.
 template <int RND>
 __host__ __device__ constexpr int quant_min_blocks() {
-  return (RND == R_RTN || RND == R_SQ16 || RND == R_AMAX) ? 4 : ((RND == R_FOS || RND == R_EDEN) ? 3 : 1);
+  return (RND == R_RTN || RND == R_SQ16 || RND == R_AMAX) ? 3 : ((RND == R_FOS || RND == R_EDEN) ? 2 : 1);
 }
-// The transposed kernel's shared-memory tile allows 6 blocks per SM; its
-// compute phase needs fewer registers, and 4 resident blocks overlap one
-// block's loads with the others' arithmetic.
+// Resident 128-thread blocks per SM of the transposed kernel: its 18.6 KB
+// tile and 64 registers allow 8, which overlap one block's loads with the
+// others' arithmetic (smaller blocks than 256 threads wait less at the
+// barrier between the two phases).
 template <int RND>
 __host__ __device__ constexpr int quant_trans_min_blocks() {
-  return (RND == R_SR || RND == R_QUEST) ? 1 : 4;
+  return (RND == R_SR || RND == R_QUEST) ? 2 : 8;
 }
 
 // Row-wise, 32 elements per lane, grid-stride over 32-element tasks.
@@ -530,6 +604,15 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
   const int64_t base0 = int64_t(blockIdx.x) * blockDim.x + (threadIdx.x & ~31);
   int64_t trow = (base0 + lane) / tpr, tct = (base0 + lane) % tpr;
   const int64_t drow = stride / tpr, dct = stride % tpr;
+  // bf16 input: the next task's 64 bytes are loaded before this task is
+  // processed, so their latency overlaps the arithmetic
+  uint4 pv[4];
+  if (LOAD == LD_ROW) {
+    const bool a0 = base0 + lane < tasks;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + (a0 ? trow * p.cols + tct * 32 : 0));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pv[i] = a0 ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+  }
   for (int64_t base = base0; base < tasks; base += stride) {
     const int64_t t = base + lane;
     const bool active = t < tasks;
@@ -539,10 +622,16 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
     if (tct >= tpr) { tct -= tpr; ++trow; }
     float x[32];
     if (LOAD == LD_ROW) {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + orow * p.cols + ocol);
       uint4 v[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = active ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 4; ++i) v[i] = pv[i];
+      {
+        const bool an = t + stride < tasks;
+        const uint4* src =
+            reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + (an ? trow * p.cols + tct * 32 : 0));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pv[i] = an ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         v[i].x ^= sm[4 * i]; v[i].y ^= sm[4 * i + 1]; v[i].z ^= sm[4 * i + 2]; v[i].w ^= sm[4 * i + 3];
@@ -579,20 +668,21 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
 
 // Transposed, 32 elements per lane: an input tile of T32Tile::ROWS rows (the
 // output rows' length covered by one block: 128, or 256 for 256-element
-// rotation blocks) x T32Tile::COLS columns (8192 elements) is staged as fp32
+// rotation blocks) x T32Tile::COLS columns (4096 elements) is staged as fp32
 // with a 4-float skew every 32 columns, so the 16-byte reads of the lanes on
 // one output row hit distinct banks.
 template <int HAD>
 struct T32Tile {
+  static constexpr int THREADS = 128;
   static constexpr int ROWS = HAD > 128 ? 256 : 128;   // input rows = output columns per block
-  static constexpr int COLS = 8192 / ROWS;               // input columns = output rows per block
+  static constexpr int COLS = THREADS * 32 / ROWS;       // input columns = output rows per block
   static constexpr int PITCH = ROWS + ROWS / 8;          // + 4 floats per 32
   static constexpr int LPR = ROWS / 32;                  // lanes per output row
 };
 __device__ __forceinline__ int t32_col(int c) { return c + 4 * (c >> 5); }
 
 template <int LOAD, int FMT, int RND, int HAD>
-__global__ void __launch_bounds__(256, quant_trans_min_blocks<RND>()) k_quant_trans32(QParams p) {
+__global__ void __launch_bounds__(T32Tile<HAD>::THREADS, quant_trans_min_blocks<RND>()) k_quant_trans32(QParams p) {
   using TT = T32Tile<HAD>;
   __shared__ Shared sh;
   __shared__ __align__(16) float tile[TT::COLS][TT::PITCH];
@@ -710,9 +800,10 @@ static __global__ void k_selftest_e2m1(unsigned long long* mismatches) {
 // E8M3 value, [2] exact_div on 2^32 hashed (dividend, divisor) pairs over the
 // whole divisor range with quotients 2^-25 .. 2^9, [3] the E4M3 decoder over
 // every non-NaN code in both byte positions, [4] the E4M3 encoder over every
-// non-negative finite fp32 value in both byte positions.
+// non-negative finite fp32 value in both byte positions, [5] the MS-EDEN
+// pseudo-scale e8m3_div6 over every non-negative fp32 value up to +inf.
 static __global__ void k_selftest_arith(unsigned long long* mismatches) {
-  unsigned long long bad[5] = {0, 0, 0, 0, 0};
+  unsigned long long bad[6] = {0, 0, 0, 0, 0, 0};
   const uint64_t stride = uint64_t(gridDim.x) * blockDim.x;
   const uint64_t tid = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const ExactDiv six = exact_div_setup(6.0f);
@@ -722,6 +813,10 @@ static __global__ void k_selftest_arith(unsigned long long* mismatches) {
     const float t1 = bitsf(uint32_t(0x7F7FFFFFull - i));
     const uint32_t c2 = e4m3x2_rtn(a, t1);
     bad[4] += (c2 & 0xFFu) != e4m3_rtn(a) || (c2 >> 8) != e4m3_rtn(t1);
+  }
+  for (uint64_t i = tid; i <= 0x7F800000ull; i += stride) {
+    const float g = bitsf(uint32_t(i));
+    bad[5] += fbits(e8m3_div6(g)) != fbits(e8m3_round(__fdiv_rn(g, 6.0f)));
   }
   for (uint64_t i = tid; i < 255ull * 8; i += stride) {   // exponent field 0..254, 3 mantissa bits
     const float pv = bitsf(uint32_t(((i >> 3) << 23) | ((i & 7) << 20)));
@@ -747,7 +842,7 @@ static __global__ void k_selftest_arith(unsigned long long* mismatches) {
     }
   }
 #pragma unroll
-  for (int k = 0; k < 5; ++k)
+  for (int k = 0; k < 6; ++k)
     if (bad[k]) atomicAdd(mismatches + k, bad[k]);
 }
 

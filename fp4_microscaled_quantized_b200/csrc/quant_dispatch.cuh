@@ -62,7 +62,7 @@ cudaError_t launch_one(const QParams& p, cudaStream_t s) {
     } else if (wide) {
       using TT = T32Tile<HAD>;
       dim3 grid(unsigned((p.in_rows + TT::ROWS - 1) / TT::ROWS), unsigned((p.in_cols + TT::COLS - 1) / TT::COLS));
-      k_quant_trans32<LOAD, FMT, RND, HAD><<<grid, 256, 0, s>>>(p);
+      k_quant_trans32<LOAD, FMT, RND, HAD><<<grid, TT::THREADS, 0, s>>>(p);
       count_launch();
     } else if constexpr (HAD <= 16 && RND != R_SQ16) {
       // inner dimension 16 mod 32: 8 elements per lane

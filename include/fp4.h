@@ -432,13 +432,15 @@ int fp4_selftest_e2m1(unsigned long long *mismatches_dev, fp4_stream_t stream);
 
 /* Device self-check of the exact shortcuts in the NVFP4 scale arithmetic
  * against CUDA's correctly rounded division and reciprocal and the E4M3
- * rounding.  ADDS mismatch counts to mismatches_dev[0..4] (5 counters, the
+ * rounding.  ADDS mismatch counts to mismatches_dev[0..5] (6 counters, the
  * caller zeroes them): [0] the corrected division by 6 over every
  * non-negative finite fp32 dividend, [1] the reciprocal of every
  * non-negative E8M3 value, [2] the corrected division by a per-tensor
  * divisor on 2^32 hashed dividend/divisor pairs, [3] the hardware E4M3
  * decoder over every non-NaN code, [4] the hardware E4M3 encoder over every
- * non-negative finite fp32 value. */
+ * non-negative finite fp32 value, [5] the MS-EDEN pseudo-scale rounding
+ * E8M3(g / 6) taken from the product with fp32(1/6) over every non-negative
+ * finite fp32 g and +inf. */
 int fp4_selftest_arith(unsigned long long *mismatches_dev, fp4_stream_t stream);
 
 /* Static description of a status code. */
