@@ -411,8 +411,9 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
           for (int cc = clo; cc <= chi; ++cc) {
             float d = __fmul_rn(e4m3_value(uint32_t(cc)), s32), inv = __frcp_rn(d);
             uint32_t wt[2];
-            enc16(xg, inv, finite_pos(d, inv), wt);
-            float e = sse16(xg, wt, d);
+            float qv[16];
+            enc16_dec(xg, inv, finite_pos(d, inv), wt, qv);   // raw codes: +-0 give the same error
+            float e = sse16q(xg, qv, d);
             if (e <= best) { best = e; bc = cc; }
           }
           s8 = uint32_t(bc);
@@ -513,13 +514,12 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
       const bool inwin = (sig2 <= tt) && (tt <= hi) && (sig2 > 0.0f);
       if (!inwin) continue;              // (an out-of-window candidate never wins)
       const float sc = pow2f(-e), d = pow2f(e);
-      uint32_t wt[4];
-      float v[32];
+      float v[32], qv[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = __fmul_rn(x[j], sc);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) wt[q] = enc8_hw(v + 8 * q);
-      const float s = __fadd_rn(sse16(x, wt, d), sse16(x + 16, wt + 2, d));
+      for (int q = 0; q < 4; ++q) (void)enc8_dec(v + 8 * q, qv + 8 * q);   // grid values of the raw codes: +-0 give the same error
+      const float s = __fadd_rn(sse16q(x, qv, d), sse16q(x + 16, qv + 16, d));
       if (s <= bs) { bs = s; be = e; }
       found = true;
     }

@@ -68,8 +68,9 @@ __device__ __forceinline__ int seed_code(float gm, float inv6) {
 // order candidates are visited in.  NaN errors never win.
 __device__ __forceinline__ void consider(const float* xg, int c, float d, float inv, float& best, int& bc) {
   uint32_t wt[2];
-  enc16_raw(xg, inv, finite_pos(d, inv), wt);
-  const float e = sse16(xg, wt, d);
+  float q[16];
+  enc16_dec(xg, inv, finite_pos(d, inv), wt, q);
+  const float e = sse16q(xg, q, d);
   if (e < best || (e == best && c > bc)) { best = e; bc = c; }
 }
 
