@@ -565,10 +565,16 @@ __device__ __forceinline__ uint32_t process32(float* x, bool active, int64_t oro
 // process the current one: RTN / amax at 3 blocks (85 registers) and
 // Four-Over-Six / MS-EDEN at 2 (128) run faster that way than at 4 / 3
 // blocks, with or without the early load (which spills at those budgets);
-// SR and QuEST keep their registers.
-template <int RND>
+// SR and QuEST keep their registers.  RTN behind a 64- to 256-point rotation
+// (shuffle stages) runs faster at 4 blocks without the early load.
+template <int RND, int HAD>
+__host__ __device__ constexpr bool row_prefetch() {
+  return !((RND == R_RTN || RND == R_SQ16) && HAD >= 64);
+}
+template <int RND, int HAD>
 __host__ __device__ constexpr int quant_min_blocks() {
-  return (RND == R_RTN || RND == R_SQ16 || RND == R_AMAX) ? 3 : ((RND == R_FOS || RND == R_EDEN) ? 2 : 1);
+  return (RND == R_RTN || RND == R_SQ16 || RND == R_AMAX) ? (row_prefetch<RND, HAD>() ? 3 : 4)
+                                                          : ((RND == R_FOS || RND == R_EDEN) ? 2 : 1);
 }
 // Resident 128-thread blocks per SM of the transposed kernel: its 18.6 KB
 // tile and 64 registers allow 8, which overlap one block's loads with the
@@ -581,7 +587,7 @@ __host__ __device__ constexpr int quant_trans_min_blocks() {
 
 // Row-wise, 32 elements per lane, grid-stride over 32-element tasks.
 template <int LOAD, int FMT, int RND, int HAD>
-__global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QParams p) {
+__global__ void __launch_bounds__(256, quant_min_blocks<RND, HAD>()) k_quant_row32(QParams p) {
   __shared__ Shared sh;
   load_signs<HAD>(sh, p);
   const int lane = threadIdx.x & 31;
@@ -606,8 +612,9 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
   const int64_t drow = stride / tpr, dct = stride % tpr;
   // bf16 input: the next task's 64 bytes are loaded before this task is
   // processed, so their latency overlaps the arithmetic
+  constexpr bool PF = LOAD == LD_ROW && row_prefetch<RND, HAD>();
   uint4 pv[4];
-  if (LOAD == LD_ROW) {
+  if (PF) {
     const bool a0 = base0 + lane < tasks;
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + (a0 ? trow * p.cols + tct * 32 : 0));
 #pragma unroll
@@ -623,14 +630,18 @@ __global__ void __launch_bounds__(256, quant_min_blocks<RND>()) k_quant_row32(QP
     float x[32];
     if (LOAD == LD_ROW) {
       uint4 v[4];
+      if (PF) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = pv[i];
-      {
+        for (int i = 0; i < 4; ++i) v[i] = pv[i];
         const bool an = t + stride < tasks;
         const uint4* src =
             reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + (an ? trow * p.cols + tct * 32 : 0));
 #pragma unroll
         for (int i = 0; i < 4; ++i) pv[i] = an ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + orow * p.cols + ocol);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = active ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
