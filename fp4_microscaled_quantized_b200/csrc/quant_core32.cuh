@@ -171,7 +171,10 @@ __device__ __forceinline__ void enc16_dec(const float* x, float inv, bool ok, ui
   }
 }
 
-// sse16 from grid values already decoded.
+// fp32 squared error of 16 elements against grid values q times d, pairwise
+// tree: e = x - fp32(q d), s = fp32(e e).  The subtraction is a scalar IEEE
+// operation: a packed subtraction of a packed product can be fused into one
+// multiply-add by the code generator, which changes the rounding.
 __device__ __forceinline__ float sse16q(const float* x, const float* q, float d) {
   float s[16];
 #pragma unroll
@@ -194,23 +197,6 @@ __device__ __forceinline__ void dec8(uint32_t w, float* q) {
     q[2 * k] = f.x;
     q[2 * k + 1] = f.y;
   }
-}
-
-// fp32 squared error of 16 elements against codes * d, pairwise tree:
-// e = x - fp32(q d), s = fp32(e e).  The subtraction is a scalar IEEE
-// operation: a packed subtraction of a packed product can be fused into one
-// multiply-add by the code generator, which changes the rounding.
-__device__ __forceinline__ float sse16(const float* x, const uint32_t* w, float d) {
-  float q[16], s[16];
-  dec8(w[0], q);
-  dec8(w[1], q + 8);
-#pragma unroll
-  for (int j = 0; j < 16; j += 2) {
-    const float2 qd = __fmul2_rn(ld2(q, j), splat2(d));
-    const float2 e = make_float2(__fsub_rn(x[j], qd.x), __fsub_rn(x[j + 1], qd.y));
-    st2(s, j, __fmul2_rn(e, e));
-  }
-  return tree16p(s);
 }
 
 // Per-lane XOR masks that apply the randomized-Hadamard signs to loaded data

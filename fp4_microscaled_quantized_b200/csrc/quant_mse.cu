@@ -4,7 +4,7 @@
 // Group step, one 32-element task (two scale groups) per thread: every
 // candidate E4M3 code c = 1..126 gives d = fp32(E4M3(c) s_T) and its correctly
 // rounded reciprocal (a per-block table, s_T being uniform), the RTN codes of
-// x * (1/d) and their fp32 squared error (sse16, the pairwise tree of
+// x * (1/d) and their fp32 squared error (sse16q, the pairwise tree of
 // fp32((x - fp32(q d))^2)); the smallest error wins, ties to the larger code.
 // Candidates that the top element's own error term already rules out are not
 // evaluated in full (top_term), and the scan below the seed stops where that
