@@ -708,7 +708,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
                                                                             // + 4 stager warps x 2 CTAs
   uint64_t* empty = full + STAGES;                                          // both: stage consumed by the MMAs
   uint64_t* sf_ld = empty + STAGES;                                         // both: this CTA's scale atoms landed
-  uint64_t* acc_full = sf_ld + STAGES;                                      // both
+  uint64_t* sf_free = sf_ld + STAGES;                                       // both: the stagers have read them
+  uint64_t* acc_full = sf_free + STAGES;                                    // both
   uint64_t* acc_empty = acc_full + 1;                                       // leader: 4 warps x 2 CTAs
   uint64_t* drain = acc_empty + 1;                                          // leader: MMAs retired
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -727,6 +728,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
       mbar_init(&full[s], 1 + 8);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_ld[s], 1);
+      mbar_init(&sf_free[s], 4);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 16);
@@ -754,10 +756,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
   if ((warp == 0 || warp == 3) && lane == 0) {
     // --------------------------------------------- producers (2 threads) --
     // Warp 0 loads the operand tiles (TMA, completing on the leader's
-    // full[s]), warp 3 this CTA's scale atoms (bulk copies, on its own
+    // full[s]), warp 3 this CTA's scale atoms (3-D TMA, on its own
     // sf_ld[s]): one thread issuing every copy of a k-tile is itself the
-    // bottleneck at this rate.  Both walk the same stages and wait for the
-    // same releases.
+    // bottleneck at this rate.  Both walk the same stages; the operands wait
+    // for the MMAs to release a stage, the scale atoms only for the stagers
+    // to have read its slot, so their copies run up to a ring ahead.
     const bool operands = warp == 0;
     int s = 0;
     uint32_t ph = 0;
@@ -773,7 +776,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
       const bool load_a = ra < nrb_a, load_b = rb < nrb_b;
       const uint32_t op_bytes = uint32_t((a_halves + b_halves) * A_BYTES);
       for (int kt = 0; kt < nk; ++kt) {
-        if (!wait_c(&empty[s], ph ^ 1, abort_flag, st)) break;
+        // operands wait for the MMAs to release the stage; scale atoms only for
+        // the stagers to have read the slot (they run up to a ring ahead)
+        if (!wait_c(operands ? &empty[s] : &sf_free[s], ph ^ 1, abort_flag, st)) break;
         if (operands) {
           if (leader) mbar_expect_tx(&full[s], op_bytes);
           if (load_a) tma_load_pair(sA + s * A_BYTES, &map_a, kt * (BK / 2), int(ra * 128), &full[s]);
@@ -852,9 +857,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
   } else if (wg == 1) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_STAGE));
     // ------------------------------------------- scale factors -> TMEM --
-    // Scale buffer s is free once stage s's scale atoms have landed: the
-    // producer issued their copies after the MMAs that last read buffer s
-    // released the stage.  Each stager warp arrives on the leader's full[s].
+    // Each stager warp reads stage s's scale atoms once they have landed,
+    // frees the slot for the next round's copies (sf_free), waits for the
+    // MMAs that last read scale TMEM buffer s to retire (empty), writes the
+    // buffer and arrives on the leader's full[s].
     const int q = warp & 3;
     int s = 0;
     uint32_t ph = 0;
@@ -879,6 +885,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PTHREADS, 1)
             vb[o] = y.x; vb[o + 1] = y.y; vb[o + 2] = y.z; vb[o + 3] = y.w;
           }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_free[s]);     // the slot may be refilled
+        // scale TMEM buffer s is free once the MMAs of its previous round retired
+        const bool e = wait_c(&empty[s], ph ^ 1, abort_flag, p.status);
+        if (__any_sync(0xFFFFFFFFu, !e)) { ok = false; break; }
+        tc_fence_after();
         const uint32_t base = tmem + (uint32_t(q * 32) << 16) + SF_COL + SF_BUF_COLS * uint32_t(s);
         asm volatile(
             "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(base),
