@@ -523,6 +523,13 @@ def sweep_cases(api):
     # the MSE-optimal scale search (fp4_quantize_mse) with 0 and 2 alternations
     out.append(("nvfp4-mse-i0-h0", api.NVFP4, "mse0", 0, False))
     out.append(("nvfp4-mse-i2-h0", api.NVFP4, "mse2", 0, False))
+    # forward-only transforms: a DCT-II / DST-II block transform (fp32 out)
+    # quantised by fp4_quantize_f32, and MXFP4 with fitted scales
+    for kind, k, fmt, fname in (("dct2", 32, api.NVFP4, "nvfp4"), ("dct2", 128, api.NVFP4, "nvfp4"),
+                                ("dst2", 256, api.MXFP4, "mxfp4")):
+        out.append(("%s-rtn-%s-k%d" % (fname, kind, k), fmt, ("xform", kind, k), k, False))
+    for had in (0, 32):
+        out.append(("mxfp4-fit-h%d" % had, api.MXFP4, ("fit",), had, False))
     return out
 
 
@@ -533,6 +540,12 @@ def sweep_bytes_per_elem(api, fmt, rnd, had):
     the amax and once per group step, writing codes and scales each time."""
     if isinstance(rnd, str):
         return 2.0 + (int(rnd[3:]) + 1) * (2.0 + 0.5 + 1.0 / 16)
+    if isinstance(rnd, tuple) and rnd[0] == "xform":
+        # bf16 read + fp32 write, then the fp32 quantiser: (amax read 4 for NVFP4) + read 4 + codes + scales
+        return 2.0 + 4.0 + (4.0 if fmt == api.NVFP4 else 0.0) + 4.0 + 0.5 + (1.0 / 16 if fmt == api.NVFP4 else 1.0 / 32)
+    if isinstance(rnd, tuple) and rnd[0] == "fit":
+        # range pass read 2, quantise pass read 2 + codes 0.5 + one level byte per 32
+        return 2.0 + 2.0 + 0.5 + 1.0 / 32
     return quant_bytes(api, fmt, rnd, had, "bf16")
 
 
@@ -570,6 +583,20 @@ def quant_sweep(args):
             if isinstance(rnd, str):
                 ws = api.alloc_workspace(api.quantize_mse_workspace_size(rows, SWEEP_COLS), dev)
                 call = lambda s, it=int(rnd[3:]): api.quantize_mse(x, it, out=out, ws=ws)  # noqa: E731
+            elif isinstance(rnd, tuple) and rnd[0] == "xform":
+                y = torch.empty((rows, SWEEP_COLS), dtype=torch.float32, device=dev)
+                ws = api.alloc_workspace(max(api.workspace_size(rows, SWEEP_COLS, fmt, api.RTN, 0), 4 * had * had), dev)
+                kind = api.XFORM_DCT2 if rnd[1] == "dct2" else api.XFORM_DST2
+
+                def call(s, kind=kind, y=y, ws=ws, out=out):
+                    api.block_transform(x, kind, had, out=y, ws=ws)
+                    api.quantize_f32(y, fmt, api.RTN, s, 1, linear=False, out=out, ws=ws)
+            elif isinstance(rnd, tuple) and rnd[0] == "fit":
+                ws = api.alloc_workspace(api.quantize_mx_fit_workspace_size(), dev)
+                fit = api.FitTensor(torch.empty((rows, SWEEP_COLS // 2), dtype=torch.uint8, device=dev),
+                                    torch.empty((rows, SWEEP_COLS // 32), dtype=torch.uint8, device=dev),
+                                    torch.empty((256,), dtype=torch.float32, device=dev))
+                call = lambda s, h=had, ws=ws, fit=fit: api.quantize_mx_fit(x, h, ws=ws, out=fit)  # noqa: E731
             else:
                 ws = api.alloc_workspace(api.workspace_size(rows, SWEEP_COLS, fmt, rnd, had), dev)
                 call = lambda s: api.quantize(x, fmt, rnd, had, rand, s, 0, 1, out=out, ws=ws)  # noqa: E731

@@ -324,8 +324,16 @@ class FitTensor:
     table: torch.Tensor
 
 
-def quantize_mx_fit(x, had_block=0, ws=None):
-    """fp4_quantize_mx_fit (MXFP4-dagger) of a bf16 CUDA tensor."""
+def quantize_mx_fit_workspace_size():
+    lib = load()
+    lib.fp4_quantize_mx_fit_workspace_size.restype = ctypes.c_size_t
+    lib.fp4_quantize_mx_fit_workspace_size.argtypes = []
+    return int(lib.fp4_quantize_mx_fit_workspace_size())
+
+
+def quantize_mx_fit(x, had_block=0, ws=None, out=None):
+    """fp4_quantize_mx_fit (MXFP4-dagger) of a bf16 CUDA tensor (into `out`,
+    a FitTensor of the right shapes, when given)."""
     lib = load()
     lib.fp4_quantize_mx_fit_workspace_size.restype = ctypes.c_size_t
     lib.fp4_quantize_mx_fit_workspace_size.argtypes = []
@@ -335,9 +343,9 @@ def quantize_mx_fit(x, had_block=0, ws=None):
                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
     assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
     rows, cols = x.shape
-    ft = FitTensor(torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device),
-                   torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device),
-                   torch.empty((256,), dtype=torch.float32, device=x.device))
+    ft = out if out is not None else FitTensor(torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device),
+                                               torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device),
+                                               torch.empty((256,), dtype=torch.float32, device=x.device))
     if ws is None:
         ws = alloc_workspace(lib.fp4_quantize_mx_fit_workspace_size(), x.device)
     _check(f(_ptr(x), rows, cols, had_block, _ptr(ft.codes), _ptr(ft.levels), _ptr(ft.table), _ptr(ws), ws.numel(),

@@ -38,3 +38,17 @@ def test_sweep_bytes_per_element():
     assert bench.sweep_bytes_per_elem(api, api.MXFP4, api.QUEST, 32) == pytest.approx(2.53125 + 0.125)
     assert bench.sweep_bytes_per_elem(api, api.NVFP4, api.MS_EDEN, 128) == pytest.approx(2.875)
     assert bench.sweep_bytes_per_elem(api, api.NVFP4, "mse2", 0) == pytest.approx(2 + 3 * 2.5625)
+    # transform (bf16 read, fp32 write) + fp32 quantiser (NVFP4: amax read, read, codes, scales)
+    assert bench.sweep_bytes_per_elem(api, api.NVFP4, ("xform", "dct2", 128), 128) == pytest.approx(14.5625)
+    assert bench.sweep_bytes_per_elem(api, api.MXFP4, ("xform", "dst2", 256), 256) == pytest.approx(10.53125)
+    # MXFP4 with fitted scales: range pass + quantise pass
+    assert bench.sweep_bytes_per_elem(api, api.MXFP4, ("fit",), 0) == pytest.approx(4.53125)
+
+
+def test_sweep_cases_are_unique_and_cover_the_forward_only_variants():
+    from fp4_microscaled_quantized_b200 import api
+    names = [c[0] for c in bench.sweep_cases(api)]
+    assert len(names) == len(set(names))
+    for n in ("nvfp4-rtn-dct2-k32", "nvfp4-rtn-dct2-k128", "mxfp4-rtn-dst2-k256", "mxfp4-fit-h0", "mxfp4-fit-h32",
+              "nvfp4-mse-i0-h0", "nvfp4-eden-h128"):
+        assert n in names
