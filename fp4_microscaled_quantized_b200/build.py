@@ -26,7 +26,7 @@ COMMON = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcom
 def _flags(src):
     extra = []
     name = os.path.basename(src)
-    if name.startswith("quant") or name == "capi.cu":
+    if name.startswith("quant") or name in ("capi.cu", "transform.cu"):
         extra += ["-fmad=false"]
     return COMMON + extra
 

@@ -52,46 +52,64 @@ __global__ void k_dense_matrix(float* m, int k, int kind) {
   }
 }
 
-// One CTA: R rows x I outputs of one k-block (I = min(k, 32), R = 256 / I);
-// the I matrix rows and the R input rows are staged in shared memory with a
-// one-float skew so the 32 lanes' matrix reads hit distinct banks.
+// One CTA: R rows x I outputs of one k-block (I = min(k, 32), R = 2 x 256 / I);
+// each thread computes output i of two rows together (the products as one f32x2
+// multiply, each half rounded as the scalar product).  The I matrix rows are
+// staged in shared memory with a one-float skew so the 32 lanes' matrix reads
+// hit distinct banks; the input is staged transposed, the two rows of a thread
+// side by side (a 2-float skew per column), so a lane reads both rows' x_j in
+// one 8-byte load.  Tree levels above the first add sums only and run two rows
+// per instruction; the first level, whose operands are products, is scalar (a
+// packed add of packed products may be contracted into a multiply-add).
 template <int K>
-__global__ void __launch_bounds__(256) k_dense_transform(const uint16_t* __restrict__ x, float* __restrict__ y,
-                                                         const float* __restrict__ m, int64_t rows, int64_t cols) {
-  constexpr int I = K < 32 ? K : 32, R = 256 / I, P = K + 1, DEPTH = 9;
+constexpr int dense_threads() { return K == 256 ? 128 : 256; }   // 256-blocks: the staging fits 48 KB
+
+template <int K>
+__global__ void __launch_bounds__(dense_threads<K>()) k_dense_transform(const uint16_t* __restrict__ x,
+                                                                      float* __restrict__ y,
+                                                                      const float* __restrict__ m, int64_t rows,
+                                                                      int64_t cols) {
+  constexpr int NT = dense_threads<K>();
+  constexpr int I = K < 32 ? K : 32, RP = NT / I, R = 2 * RP, P = K + 1, XP = R + 2, DEPTH = 9;
   constexpr int ROOT = K == 16 ? 4 : K == 32 ? 5 : K == 64 ? 6 : K == 128 ? 7 : 8;   // log2 K
   __shared__ float sm[I][P];
-  __shared__ float sx[R][P];
+  __shared__ __align__(8) float sx[K][XP];          // sx[j][r] = x[r0 + r][c0 + j]
   const int64_t r0 = int64_t(blockIdx.x) * R, c0 = int64_t(blockIdx.y) * K;
   const int i0 = blockIdx.z * I;
-  for (int t = threadIdx.x; t < I * K; t += 256) sm[t / K][t % K] = m[(i0 + t / K) * K + t % K];
-  for (int t = threadIdx.x; t < R * K; t += 256) {
+  for (int t = threadIdx.x; t < I * K; t += NT) sm[t / K][t % K] = m[(i0 + t / K) * K + t % K];
+  for (int t = threadIdx.x; t < R * K; t += NT) {
     const int64_t r = r0 + t / K;
-    sx[t / K][t % K] = r < rows ? __uint_as_float(uint32_t(x[r * cols + c0 + t % K]) << 16) : 0.0f;
+    sx[t % K][t / K] = r < rows ? __uint_as_float(uint32_t(x[r * cols + c0 + t % K]) << 16) : 0.0f;
   }
   __syncthreads();
-  const int i = threadIdx.x % I, r = threadIdx.x / I;
-  float stack[DEPTH];
+  const int i = threadIdx.x % I, rp = threadIdx.x / I;
+  float2 stack[DEPTH];
 #pragma unroll
   for (int j = 0; j < K; ++j) {
-    float v = __fmul_rn(sm[i][j], sx[r][j]);
+    float2 v = __fmul2_rn(make_float2(sm[i][j], sm[i][j]), *reinterpret_cast<const float2*>(&sx[j][2 * rp]));
     int level = 0;
+    if (j & 1) {                          // leaf j closes the subtrees of its trailing one bits
+      v = make_float2(__fadd_rn(stack[0].x, v.x), __fadd_rn(stack[0].y, v.y));
+      level = 1;
 #pragma unroll
-    for (int b = 0; b < DEPTH; ++b) {   // leaf j closes the subtrees of its trailing one bits
-      if (((j >> b) & 1) == 0) break;
-      v = __fadd_rn(stack[b], v);
-      level = b + 1;
+      for (int b = 1; b < DEPTH; ++b) {
+        if (((j >> b) & 1) == 0) break;
+        v = __fadd2_rn(stack[b], v);
+        level = b + 1;
+      }
     }
     stack[level] = v;
   }
-  if (r0 + r < rows) y[(r0 + r) * cols + c0 + i0 + i] = stack[ROOT];
+  const int64_t ra = r0 + 2 * rp;
+  if (ra < rows) y[ra * cols + c0 + i0 + i] = stack[ROOT].x;
+  if (ra + 1 < rows) y[(ra + 1) * cols + c0 + i0 + i] = stack[ROOT].y;
 }
 
 template <int K>
 cudaError_t launch_dense(const uint16_t* x, float* y, const float* m, int64_t rows, int64_t cols, cudaStream_t s) {
-  constexpr int I = K < 32 ? K : 32, R = 256 / I;
+  constexpr int I = K < 32 ? K : 32, R = 2 * dense_threads<K>() / I;
   const dim3 grid(unsigned((rows + R - 1) / R), unsigned(cols / K), unsigned(K / I));
-  k_dense_transform<K><<<grid, 256, 0, s>>>(x, y, m, rows, cols);
+  k_dense_transform<K><<<grid, dense_threads<K>(), 0, s>>>(x, y, m, rows, cols);
   count_launch();
   return cudaGetLastError();
 }
