@@ -2,8 +2,9 @@
 
 Each ``csrc/*.cu`` compiles to an object in ``_build/`` (in parallel, rebuilt
 when a source or header is newer), then all link into one shared library next
-to this file.  The quantiser sources build with ``-fmad=false`` so no fp32
-multiply-add is ever contracted (the arithmetic contract with the oracle).
+to this file.  The quantiser, C-ABI and block-transform sources build with
+``-fmad=false`` so no fp32 multiply-add is ever contracted (the arithmetic
+contract with the oracle).
 """
 import concurrent.futures as cf
 import glob
