@@ -1,6 +1,7 @@
-"""Pins of the oracle's MXFP4 RTN and stochastic-rounding errors to their
-expected values on Gaussian data, computed by numerical integration from
-the format's definition alone (no oracle code): groups of 32 iid N(0, 1)
+"""Pins of the oracle's MXFP4 RTN and stochastic-rounding errors, and of its
+NVFP4 RTN error, to their expected values on Gaussian data, computed by
+numerical integration from the formats' definitions alone (no oracle code).
+MXFP4: groups of 32 iid N(0, 1)
 values (the same after an orthonormal 32-point Hadamard, which maps iid
 N(0, 1) to iid N(0, 1)), the shared scale 2^(floor(log2 M) - 2) of the
 group maximum M (the OCP rule of the Quartet and Bridging-the-Gap pages),
@@ -15,6 +16,10 @@ element:
   no clipping) and the 4/3 carried back: unbiased, with conditional
   variance (4 s / 3)^2 (v - lo)(hi - v) between the neighbouring grid
   points lo <= v <= hi.
+NVFP4 RTN: groups of 16, the tensor scale s_T = amax / (6 x 256) of the
+sample, the group scale d = s_T x E4M3(M / (6 s_T)) (round to nearest,
+3 mantissa bits), elements rounded to the grid times d (saturating at 6 d,
+which the max element can exceed when E4M3 rounds its scale down).
 The oracle's Monte Carlo means over 2^20 elements must match within their
 sampling error (1%)."""
 import math
@@ -106,3 +111,38 @@ def test_mxfp4_sr_mean_squared_error_is_the_integral():
     got = _mse(qn.mxfp4_sr(x, 5, 1), x)
     assert abs(got - want) <= 0.01 * want
     assert want > _expected_mse("rtn")                   # the ordering the Quartet page states
+
+
+def _nvfp4_rtn_expected_mse(s_t):
+    def dens(m):
+        return 16.0 * _cdf2(m) ** 15 * 2.0 * _phi(m)
+
+    def piece(a, b, d):
+        def per_group(m):
+            pts = [0.0] + [p for p in list(MIDS * d) + [6.0 * d] if 0.0 < p < m] + [m]
+            inner = sum(integrate.quad(lambda y: _rtn_err(y, d) * 2.0 * _phi(y), lo, hi, epsabs=1e-14)[0]
+                        for lo, hi in zip(pts[:-1], pts[1:]))
+            return (_rtn_err(m, d) + 15.0 * inner / _cdf2(m)) / 16.0
+        return integrate.quad(lambda m: dens(m) * per_group(m), a, b, epsabs=1e-13, limit=100)[0]
+
+    # every normal E4M3 value and the interval of t = M / (6 s_T) that rounds to it
+    vals = sorted({2.0 ** e * (1.0 + mm / 8.0) for e in range(-6, 9) for mm in range(8) if 2.0 ** e * (1.0 + mm / 8.0) <= 448.0})
+    total = 0.0
+    for i, v in enumerate(vals):
+        t_lo = 0.5 * (vals[i - 1] + v) if i else v
+        t_hi = 0.5 * (v + vals[i + 1]) if i + 1 < len(vals) else 2.0 * v
+        a, b = 6.0 * s_t * t_lo, min(6.0 * s_t * t_hi, 9.0)
+        if a >= b or b < 0.05:                           # P(M < 0.05) < 1e-20 for 16 values
+            continue
+        total += piece(a, b, v * s_t)
+    return total
+
+
+def test_nvfp4_rtn_mean_squared_error_is_the_integral():
+    x = _gauss(13)
+    amax = float(np.max(np.abs(x)))
+    s_t = float(np.float32(np.float32(amax) / np.float32(6.0 * 256.0)))
+    want = _nvfp4_rtn_expected_mse(s_t)
+    got = _mse(qn.nvfp4_rtn(x), x)
+    assert abs(got - want) <= 0.01 * want
+
