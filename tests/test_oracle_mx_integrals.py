@@ -19,7 +19,9 @@ element:
 NVFP4 RTN: groups of 16, the tensor scale s_T = amax / (6 x 256) of the
 sample, the group scale d = s_T x E4M3(M / (6 s_T)) (round to nearest,
 3 mantissa bits), elements rounded to the grid times d (saturating at 6 d,
-which the max element can exceed when E4M3 rounds its scale down).
+which the max element can exceed when E4M3 rounds its scale down).  NVFP4
+SR: the 16/17 guard in both scales, unbiased SR of y / d (variance
+d^2 (v - lo)(hi - v)), no clipping.
 The oracle's Monte Carlo means over 2^20 elements must match within their
 sampling error (1%)."""
 import math
@@ -113,25 +115,39 @@ def test_mxfp4_sr_mean_squared_error_is_the_integral():
     assert want > _expected_mse("rtn")                   # the ordering the Quartet page states
 
 
-def _nvfp4_rtn_expected_mse(s_t):
+def _nv_sr_err(y, d):
+    """Expected squared error of unbiased SR of y / d on the grid (no clipping), times d^2."""
+    v = y / d
+    i = min(int(np.searchsorted(GRID, v, side="right")) - 1, len(GRID) - 2)
+    lo, hi = GRID[i], GRID[i + 1]
+    return d * d * (v - lo) * (hi - v)
+
+
+def _nvfp4_expected_mse(s_t, group_div, kind):
+    """Groups of 16: the group scale d = s_T x E4M3(M / (group_div s_T)); RTN
+    (saturating at 6 d) or SR (the 16/17 guard keeps y / d within 6)."""
+    err = _rtn_err if kind == "rtn" else _nv_sr_err
+
     def dens(m):
         return 16.0 * _cdf2(m) ** 15 * 2.0 * _phi(m)
 
     def piece(a, b, d):
         def per_group(m):
-            pts = [0.0] + [p for p in list(MIDS * d) + [6.0 * d] if 0.0 < p < m] + [m]
-            inner = sum(integrate.quad(lambda y: _rtn_err(y, d) * 2.0 * _phi(y), lo, hi, epsabs=1e-14)[0]
+            marks = list(MIDS * d) + [6.0 * d] if kind == "rtn" else list(GRID[1:-1] * d)
+            pts = [0.0] + [p for p in marks if 0.0 < p < m] + [m]
+            inner = sum(integrate.quad(lambda y: err(y, d) * 2.0 * _phi(y), lo, hi, epsabs=1e-14)[0]
                         for lo, hi in zip(pts[:-1], pts[1:]))
-            return (_rtn_err(m, d) + 15.0 * inner / _cdf2(m)) / 16.0
+            return (err(m, d) + 15.0 * inner / _cdf2(m)) / 16.0
         return integrate.quad(lambda m: dens(m) * per_group(m), a, b, epsabs=1e-13, limit=100)[0]
 
-    # every normal E4M3 value and the interval of t = M / (6 s_T) that rounds to it
-    vals = sorted({2.0 ** e * (1.0 + mm / 8.0) for e in range(-6, 9) for mm in range(8) if 2.0 ** e * (1.0 + mm / 8.0) <= 448.0})
+    # every normal E4M3 value and the interval of t = M / (group_div s_T) that rounds to it
+    vals = sorted({2.0 ** e * (1.0 + mm / 8.0) for e in range(-6, 9) for mm in range(8)
+                   if 2.0 ** e * (1.0 + mm / 8.0) <= 448.0})
     total = 0.0
     for i, v in enumerate(vals):
         t_lo = 0.5 * (vals[i - 1] + v) if i else v
         t_hi = 0.5 * (v + vals[i + 1]) if i + 1 < len(vals) else 2.0 * v
-        a, b = 6.0 * s_t * t_lo, min(6.0 * s_t * t_hi, 9.0)
+        a, b = group_div * s_t * t_lo, min(group_div * s_t * t_hi, 9.0)
         if a >= b or b < 0.05:                           # P(M < 0.05) < 1e-20 for 16 values
             continue
         total += piece(a, b, v * s_t)
@@ -140,9 +156,20 @@ def _nvfp4_rtn_expected_mse(s_t):
 
 def test_nvfp4_rtn_mean_squared_error_is_the_integral():
     x = _gauss(13)
-    amax = float(np.max(np.abs(x)))
-    s_t = float(np.float32(np.float32(amax) / np.float32(6.0 * 256.0)))
-    want = _nvfp4_rtn_expected_mse(s_t)
+    amax = np.float32(np.max(np.abs(x)))
+    s_t = float(np.float32(amax / np.float32(6.0 * 256.0)))
+    want = _nvfp4_expected_mse(s_t, 6.0, "rtn")
     got = _mse(qn.nvfp4_rtn(x), x)
     assert abs(got - want) <= 0.01 * want
 
+
+def test_nvfp4_sr_mean_squared_error_is_the_integral():
+    """The Quartet II page's standard NVFP4 SR: s_T = amax / (6 x 16/17 x 448),
+    group scale E4M3(M / (6 x 16/17 x s_T))."""
+    x = _gauss(14)
+    amax = np.float32(np.max(np.abs(x)))
+    g = 6.0 * 16.0 / 17.0
+    s_t = float(np.float32(amax / np.float32(g * 448.0)))
+    want = _nvfp4_expected_mse(s_t, float(np.float32(g)), "sr")
+    got = _mse(qn.nvfp4_sr(x, 3, 1), x)
+    assert abs(got - want) <= 0.01 * want
