@@ -343,6 +343,10 @@ def quantize_mx_fit(x, had_block=0, ws=None, out=None):
                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
     assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
     rows, cols = x.shape
+    if out is not None:
+        assert (tuple(out.codes.shape) == (rows, cols // 2) and tuple(out.levels.shape) == (rows, cols // 32)
+                and tuple(out.table.shape) == (256,) and out.table.dtype == torch.float32
+                and out.codes.dtype == torch.uint8 and out.levels.dtype == torch.uint8), "out: wrong shapes or types"
     ft = out if out is not None else FitTensor(torch.empty((rows, cols // 2), dtype=torch.uint8, device=x.device),
                                                torch.empty((rows, cols // 32), dtype=torch.uint8, device=x.device),
                                                torch.empty((256,), dtype=torch.float32, device=x.device))
