@@ -288,6 +288,7 @@ def block_transform(x, kind, block, out=None, ws=None):
     assert x.dtype == torch.bfloat16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
     if out is None:
         out = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    assert out.shape == x.shape and out.dtype == torch.float32 and out.is_contiguous(), "out: fp32, x's shape"
     if ws is None:
         ws = alloc_workspace(lib.fp4_block_transform_workspace_size(block), x.device)
     _check(f(_ptr(x), _ptr(out), x.shape[0], x.shape[1], kind, block, _ptr(ws), ws.numel(), _stream()),
