@@ -111,6 +111,13 @@ def _check(st, what):
         raise Fp4Error(st, what)
 
 
+def _check_out(t, shape, what):
+    """A caller-given output must be a contiguous tensor of the shape the C
+    call writes (the C ABI sees only its pointer)."""
+    assert tuple(t.shape) == tuple(shape) and t.is_contiguous(), "%s: expected a contiguous %s tensor, got %s" % (
+        what, tuple(shape), tuple(t.shape))
+
+
 @dataclass
 class QTensor:
     """A quantised tensor in device memory (rows x cols, groups along cols)."""
@@ -225,6 +232,7 @@ def dequantize(qt, out_dtype=torch.float32, out=None):
     f.argtypes = [ctypes.POINTER(fp4_qtensor), ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p]
     if out is None:
         out = torch.empty((qt.rows, qt.cols), dtype=out_dtype, device=qt.codes.device)
+    _check_out(out, (qt.rows, qt.cols), "dequantize out")
     code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
     cs = qt.c_struct()
     _check(f(ctypes.byref(cs), _ptr(out), code, _stream()), "fp4_dequantize")
@@ -368,6 +376,7 @@ def dequantize_mx_fit(ft, out=None):
     rows, cols = ft.codes.shape[0], ft.codes.shape[1] * 2
     if out is None:
         out = torch.empty((rows, cols), dtype=torch.float32, device=ft.codes.device)
+    _check_out(out, (rows, cols), "dequantize_mx_fit out")
     _check(f(_ptr(ft.codes), _ptr(ft.levels), _ptr(ft.table), rows, cols, _ptr(out), _stream()),
            "fp4_dequantize_mx_fit")
     return out
@@ -396,6 +405,7 @@ def gemm(A, B, out_dtype=torch.float32, mask=None, inverse_had=0, out=None):
     lib = load()
     if out is None:
         out = torch.empty((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
+    _check_out(out, (A.rows, B.rows), "gemm out")
     code = {torch.float32: 0, torch.bfloat16: 1}[out.dtype]
     ca, cb = A.c_struct(), B.c_struct()
     st = lib.fp4_gemm(ctypes.byref(ca), ctypes.byref(cb), _ptr(out), code, _ptr(mask),
@@ -456,6 +466,7 @@ def linear_fwd(X, W, r, seed=0, ctx=None, Y=None, ws=None):
         ctx = alloc_ctx(r, M, N, K, X.device)
     if Y is None:
         Y = torch.empty((M, N), dtype=_DT[r.out_y], device=X.device)
+    _check_out(Y, (M, N), "linear_fwd Y")
     if ws is None:
         ws = linear_workspace(r, M, N, K, False, X.device)
     c = ctx.c_struct()
@@ -475,6 +486,10 @@ def linear_bwd(dY, ctx, step_seed, dX=None, dW=None, ws=None, want_dx=True, want
         dX = torch.empty((M, K), dtype=_DT[r.out_dx], device=dY.device)
     if want_dw and dW is None:
         dW = torch.empty((N, K), dtype=_DT[r.out_dw], device=dY.device)
+    if want_dx:
+        _check_out(dX, (M, K), "linear_bwd dX")
+    if want_dw:
+        _check_out(dW, (N, K), "linear_bwd dW")
     if ws is None:
         ws = linear_workspace(r, M, N, K, True, dY.device)
     c = ctx.c_struct()

@@ -243,3 +243,21 @@ def test_transform_and_fit_argument_checks(lib):
     assert mf(FAKE, 8, 64, 0, FAKE, FAKE, FAKE, FAKE, 100, None) == WORKSPACE
     assert mf(FAKE, 8, 64, 0, None, FAKE, FAKE, FAKE, 4096, None) == INVALID
     assert mf(FAKE + 2, 8, 64, 0, FAKE, FAKE, FAKE, FAKE, 4096, None) == ALIGNMENT
+
+
+def test_binding_rejects_outputs_of_the_wrong_shape():
+    """The C ABI sees only an output's pointer, so the binding checks a
+    caller-given output's shape before the call (no device work here)."""
+    import torch
+    from fp4_microscaled_quantized_b200 import api
+
+    class Fake:
+        rows, cols = 4, 64
+        codes = torch.empty((4, 32), dtype=torch.uint8)
+
+    with pytest.raises(AssertionError):
+        api.gemm(Fake(), Fake(), out=torch.empty((4, 5)))
+    with pytest.raises(AssertionError):
+        api.dequantize(Fake(), out=torch.empty((4, 32)))
+    with pytest.raises(AssertionError):
+        api.dequantize(Fake(), out=torch.empty((64, 4)).t())          # right shape, not contiguous
